@@ -1,0 +1,240 @@
+"""Seeded synthetic workloads for block-sparse causal prefill attention.
+
+This module draws the random inputs that the five workloads are described with and casts
+them to the storage types the kernels read (bf16, or e4m3 with per-head absmax scales).
+It holds none of the method's own arithmetic (no pooling, scoring, thresholding or
+attention), so it can feed both the CUDA path and the fp64 oracle without coupling them.
+
+Workloads (sizes as the attention layers of long-context prefill are described in
+"FlashPrefill V2: Block-Sparse Prefill Attention for Long-Context LLM Serving", Abstract,
+and "FlashPrefill: Instantaneous Pattern Discovery and Thresholding ...", technical
+summary section 4):
+
+* ``tiny``     one sequence, L=2048, Hq=Hkv=4, d=64, block 64, Q,K,V ~ N(0,1).
+* ``llama32k`` one sequence, L=32768, Hq=32, Hkv=8, d=128, block 128. Q,K ~ N(0,1)/d^0.25
+               with planted "vertical" keys: at 64 seeded token positions every KV head's
+               key gets += 3u, and every query gets += u (u one seeded unit vector).
+* ``llama128k`` the same at L=131072 plus a local band: per KV head g a slowly drifting
+               stationary random walk w_g[t] (AR(1), unit variance per coordinate) is
+               added, times BAND_AMPLITUDE, to K[t, g] and to Q[t, h] of the query heads
+               h that read g. V ~ N(0,1).
+* ``fp8_128k`` the ``llama128k`` tensors quantised per head to e4m3 (scale = absmax/448).
+* ``paged``    8 requests, lengths uniform in [4096, 65536], each drawn with the
+               ``llama128k`` recipe under its own seed; K/V stored in 64-token pages
+               whose physical order is a seeded random permutation.
+
+The vertical, slash (diagonal band) and spatially contiguous patterns these stand in
+for are the ones pattern discovery targets ("FlashPrefill: Instantaneous Pattern
+Discovery ...", technical summary section 2.A).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import torch
+
+# Local-band recipe, frozen after a one-off calibration of the ``llama128k`` workload
+# (block 128, alpha 0.1): mean kept-block density lands in the 5-10 % range that the
+# 128K workload is specified with (90-95 % block sparsity); measured 7.55 % at seed 1237
+# on one KV-head group.
+BAND_AMPLITUDE = 0.60          # c: added term is c * w_g[t]
+BAND_CORR_TOKENS = 5120.0      # AR(1) correlation length tau: rho = exp(-1/tau)
+VERTICAL_COUNT = 64
+VERTICAL_GAIN = 3.0
+E4M3_MAX = 448.0
+
+_CHUNK = 1 << 22
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    seqlens: tuple            # per-request token counts (one entry for a single sequence)
+    Hq: int
+    Hkv: int
+    d: int
+    block: int
+    alpha: float = 0.1
+    dtype: str = "bf16"       # storage type of Q/K/V: "bf16" or "e4m3"
+    structure: str = "iid"    # "iid", "vertical" or "band"
+    page_size: int = 0        # 0: contiguous K/V; else paged K/V cache with this page size
+
+    @property
+    def total_tokens(self) -> int:
+        return int(sum(self.seqlens))
+
+    @property
+    def batch(self) -> int:
+        return len(self.seqlens)
+
+
+def paged_lengths(seed: int, n: int = 8, lo: int = 4096, hi: int = 65536) -> tuple:
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 77])))
+    return tuple(int(x) for x in rng.integers(lo, hi + 1, size=n))
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", (2048,), 4, 4, 64, 64, structure="iid"),
+    "llama32k": Workload("llama32k", (32768,), 32, 8, 128, 128, structure="vertical"),
+    "llama128k": Workload("llama128k", (131072,), 32, 8, 128, 128, structure="band"),
+    "fp8_128k": Workload("fp8_128k", (131072,), 32, 8, 128, 128, dtype="e4m3",
+                         structure="band"),
+    "paged": Workload("paged", paged_lengths(1234 + 5), 32, 8, 128, 128, structure="band",
+                      page_size=64),
+}
+
+DEFAULT_SEEDS = {"tiny": 1235, "llama32k": 1236, "llama128k": 1237, "fp8_128k": 1237,
+                 "paged": 1239}
+
+
+def _normal(seed_seq: np.random.SeedSequence, shape) -> np.ndarray:
+    """Standard normals in float32, drawn in fixed-size chunks with spawned seeds so
+    the result does not depend on the thread count."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float32)
+    nchunk = max(1, (n + _CHUNK - 1) // _CHUNK)
+    seeds = seed_seq.spawn(nchunk)
+
+    def fill(i):
+        lo, hi = i * _CHUNK, min(n, (i + 1) * _CHUNK)
+        np.random.Generator(np.random.PCG64(seeds[i])).standard_normal(
+            out=out[lo:hi], dtype=np.float32)
+
+    with ThreadPoolExecutor(8) as ex:
+        list(ex.map(fill, range(nchunk)))
+    return out.reshape(shape)
+
+
+def _ar1(seed_seq, T: int, ncomp: int, tau: float) -> np.ndarray:
+    """Stationary AR(1) walk x_t = rho x_{t-1} + sqrt(1-rho^2) e_t, x_0 = e_0, float32."""
+    from scipy.signal import lfilter
+    rho = math.exp(-1.0 / tau)
+    e = _normal(seed_seq, (T, ncomp)).astype(np.float64)
+    e[1:] *= math.sqrt(1.0 - rho * rho)
+    return lfilter([1.0], [1.0, -rho], e, axis=0).astype(np.float32)
+
+
+def _one_sequence(w: Workload, L: int, seed_seq: np.random.SeedSequence):
+    """Float32 Q [L,Hq,d], K [L,Hkv,d], V [L,Hkv,d] for one request."""
+    s_q, s_k, s_v, s_u, s_pos, s_band = seed_seq.spawn(6)
+    Hq, Hkv, d = w.Hq, w.Hkv, w.d
+    q = _normal(s_q, (L, Hq, d))
+    k = _normal(s_k, (L, Hkv, d))
+    v = _normal(s_v, (L, Hkv, d))
+    if w.structure == "iid":
+        return q, k, v
+    inv = np.float32(1.0 / d ** 0.25)
+    q *= inv
+    k *= inv
+    u = _normal(s_u, (d,)).astype(np.float64)
+    u = (u / np.linalg.norm(u)).astype(np.float32)
+    pos = np.random.Generator(np.random.PCG64(s_pos)).choice(
+        L, size=min(VERTICAL_COUNT, L), replace=False)
+    k[pos] += VERTICAL_GAIN * u
+    q += u
+    if w.structure == "band":
+        G = Hq // Hkv
+        band_seeds = s_band.spawn(Hkv)
+        for g in range(Hkv):
+            wg = _ar1(band_seeds[g], L, d, BAND_CORR_TOKENS) * np.float32(BAND_AMPLITUDE)
+            k[:, g, :] += wg
+            q[:, g * G:(g + 1) * G, :] += wg[:, None, :]
+    return q, k, v
+
+
+def quantize_e4m3(x: torch.Tensor, head_dim: int = 1):
+    """Per-head absmax/448 scales and the e4m3 codes (round to nearest even, clamped).
+
+    x: float32 [T, H, d]. Returns (codes float8_e4m3fn [T,H,d], scale float32 [H])."""
+    amax = x.abs().amax(dim=(0, 2)).clamp_min(1e-12)
+    scale = (amax / E4M3_MAX).to(torch.float32)
+    y = (x / scale[None, :, None]).clamp(-E4M3_MAX, E4M3_MAX)
+    return y.to(torch.float8_e4m3fn), scale
+
+
+@dataclasses.dataclass
+class Inputs:
+    """Host tensors for one workload. Q/K/V are in the storage dtype; ``*_scale`` are
+    per-head float32 dequantisation scales for e4m3 storage (None for bf16)."""
+    workload: Workload
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    cu_seqlens: torch.Tensor          # int32 [B+1]
+    q_scale: torch.Tensor | None = None
+    k_scale: torch.Tensor | None = None
+    v_scale: torch.Tensor | None = None
+    k_cache: torch.Tensor | None = None   # [num_pages, page, Hkv, d] (paged workloads)
+    v_cache: torch.Tensor | None = None
+    page_table: torch.Tensor | None = None  # int32 [B, max_pages]
+
+    def codes_f32(self, which: str) -> np.ndarray:
+        """The stored values (bf16 values or e4m3 codes) as float32 -- exact for both
+        storage types. Multiply by ``<which>_scale`` per head to get the real values."""
+        return getattr(self, which).to(torch.float32).numpy()
+
+    def scale_f64(self, which: str):
+        sc = getattr(self, which + "_scale")
+        return None if sc is None else sc.double().numpy()
+
+
+def make_inputs(name_or_w, seed: int | None = None, seqlens=None) -> Inputs:
+    """Draw one workload's inputs on the host. ``seqlens`` overrides the request lengths
+    (smaller parity cases keep the recipe and shrink the sizes)."""
+    w = WORKLOADS[name_or_w] if isinstance(name_or_w, str) else name_or_w
+    if seqlens is not None:
+        w = dataclasses.replace(w, seqlens=tuple(int(s) for s in seqlens))
+    if seed is None:
+        seed = DEFAULT_SEEDS.get(w.name, 1234)
+    root = np.random.SeedSequence(seed)
+    req_seeds = root.spawn(w.batch + 1)
+    qs, ks, vs = [], [], []
+    for b, L in enumerate(w.seqlens):
+        q, k, v = _one_sequence(w, L, req_seeds[b])
+        qs.append(q)
+        ks.append(k)
+        vs.append(v)
+    q = torch.from_numpy(np.concatenate(qs)) if len(qs) > 1 else torch.from_numpy(qs[0])
+    k = torch.from_numpy(np.concatenate(ks)) if len(ks) > 1 else torch.from_numpy(ks[0])
+    v = torch.from_numpy(np.concatenate(vs)) if len(vs) > 1 else torch.from_numpy(vs[0])
+    del qs, ks, vs
+    cu = torch.zeros(w.batch + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(w.seqlens, dtype=torch.int64), 0).to(torch.int32)
+    inp = Inputs(w, q, k, v, cu)
+    if w.dtype == "e4m3":
+        inp.q, inp.q_scale = quantize_e4m3(q)
+        inp.k, inp.k_scale = quantize_e4m3(k)
+        inp.v, inp.v_scale = quantize_e4m3(v)
+    else:
+        inp.q, inp.k, inp.v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    if w.page_size:
+        _page(inp, req_seeds[-1])
+    return inp
+
+
+def _page(inp: Inputs, seed_seq):
+    """Scatter K/V into ``page_size``-token pages in a seeded random physical order."""
+    w = inp.workload
+    P = w.page_size
+    npages = [(L + P - 1) // P for L in w.seqlens]
+    total = sum(npages)
+    perm = np.random.Generator(np.random.PCG64(seed_seq)).permutation(total)
+    maxp = max(npages)
+    table = torch.full((w.batch, maxp), -1, dtype=torch.int32)
+    kc = torch.zeros((total, P, w.Hkv, w.d), dtype=inp.k.dtype)
+    vc = torch.zeros((total, P, w.Hkv, w.d), dtype=inp.v.dtype)
+    logical = 0
+    cu = inp.cu_seqlens.tolist()
+    for b, L in enumerate(w.seqlens):
+        for p in range(npages[b]):
+            phys = int(perm[logical])
+            logical += 1
+            table[b, p] = phys
+            lo = cu[b] + p * P
+            hi = min(cu[b] + L, lo + P)
+            kc[phys, : hi - lo] = inp.k[lo:hi]
+            vc[phys, : hi - lo] = inp.v[lo:hi]
+    inp.k_cache, inp.v_cache, inp.page_table = kc, vc, table
