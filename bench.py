@@ -1,0 +1,412 @@
+"""Benchmark of one block-sparse causal prefill-attention layer (pool + mask + attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama128k]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on a bounded sample
+
+One step = the whole path over one layer's synthetic inputs: fp_pool_qk -> fp_build_block_mask
+-> fp_sparse_prefill_attn (or the paged entry), launched through the C ABI. Inputs (Q 1 GiB,
+K and V 256 MiB each at 128K) are larger than the 126 MB L2, so steps run back to back
+without an L2 flush. Timing: CUDA events on the launching stream, W warm-up steps, then K
+timed steps bracketed by barrier + synchronize; multi-GPU runs are independent replicas
+(each rank its own layer, no collective) and report the max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import block_sparse_long_qk_b200 as fp  # noqa: E402
+from block_sparse_long_qk_b200 import synthetic as S  # noqa: E402
+
+METRIC = "128K prefill-attn ms/layer incl. mask build; executed TFLOPS & % of B200 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class Clocks:
+    """Samples nvidia-smi SM clocks and throttle reasons while the timed region runs."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def start(self):
+        def run():
+            while not self._stop.is_set():
+                try:
+                    out = subprocess.run(
+                        ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                         "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                        timeout=5).stdout.strip()
+                    if out:
+                        self.rows.append([x.strip() for x in out.split(",")])
+                except Exception:
+                    pass
+                self._stop.wait(0.2)
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if len(r) > 3 + i and r[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+class Layer:
+    """Device-resident inputs and preallocated outputs of one layer, and the step."""
+
+    def __init__(self, inp, dev):
+        w = inp.workload
+        self.w = w
+        self.dev = dev
+        self.q = inp.q.to(dev)
+        self.k = inp.k.to(dev)
+        self.v = inp.v.to(dev)
+        self.scales = {n: (None if getattr(inp, n) is None else getattr(inp, n).to(dev))
+                       for n in ("q_scale", "k_scale", "v_scale")}
+        self.paged = None
+        if w.page_size:
+            self.paged = fp.PagedKV(inp.k_cache.to(dev), inp.v_cache.to(dev),
+                                    inp.page_table.to(dev))
+            self.k = self.v = None
+        self.batch = fp.Batch.make(w.seqlens, w.block, dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.ev = []
+
+    def step(self, events=None):
+        w, b = self.w, self.batch
+        sc = self.scales
+        e = events
+        if e is not None:
+            e[0].record(self.stream)
+        qp, kp = fp.pool_qk(self.q, self.k, w.block, batch=b, q_scale=sc["q_scale"],
+                            k_scale=sc["k_scale"], paged=self.paged)
+        if e is not None:
+            e[1].record(self.stream)
+        _, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b,
+                                          mask_bits=False)
+        if e is not None:
+            e[2].record(self.stream)
+        if self.paged is not None:
+            out, _ = fp.sparse_prefill_attn_paged(self.q, self.paged, cnt, idx, b,
+                                                  q_scale=sc["q_scale"], k_scale=sc["k_scale"],
+                                                  v_scale=sc["v_scale"])
+        else:
+            out, _ = fp.sparse_prefill_attn(self.q, self.k, self.v, cnt, idx, w.block, batch=b,
+                                            q_scale=sc["q_scale"], k_scale=sc["k_scale"],
+                                            v_scale=sc["v_scale"])
+        if e is not None:
+            e[3].record(self.stream)
+        return out, cnt, idx
+
+
+def work_counts(w, cnt, idx, batch):
+    """Algorithmic and executed attention FLOPs and the kept-block density of one layer."""
+    B, d = w.block, w.d
+    cnt = cnt.long()
+    seq = torch.tensor(w.seqlens, device=cnt.device)
+    nb = (seq + B - 1) // B
+    # valid rows of each global block
+    nvalid = torch.cat([torch.clamp(L - torch.arange(n, device=cnt.device) * B, max=B)
+                        for L, n in zip(seq.tolist(), nb.tolist())])
+    blk_req = torch.repeat_interleave(torch.arange(len(w.seqlens), device=cnt.device), nb)
+    off = torch.cumsum(nb, 0) - nb
+    local = torch.arange(int(nb.sum()), device=cnt.device) - off[blk_req]
+    # kept blocks other than the diagonal are full B x n_I rectangles (earlier blocks of a
+    # request are full); the diagonal block contributes n(n+1)/2 causal pairs
+    pairs = (cnt - 1) * B * nvalid[None, :] + nvalid[None, :] * (nvalid[None, :] + 1) // 2
+    alg = 4.0 * d * float(pairs.sum())
+    executed = 4.0 * 128 * B * d * float(cnt.sum())
+    causal_blocks = float(((local + 1).sum()) * w.Hq)
+    return alg, executed, float(cnt.sum()) / causal_blocks
+
+
+def pool_mask_bytes(w):
+    eb = 1 if w.dtype == "e4m3" else 2
+    T = w.total_tokens
+    nblk = sum((L + w.block - 1) // w.block for L in w.seqlens)
+    return T * (w.Hq + w.Hkv) * w.d * eb + 2 * nblk * (w.Hq + w.Hkv) * w.d * 4
+
+
+def cpu_baseline(inp, rows_sample=32, seed=5):
+    """The fp64 oracle as it stands, on a bounded sample of the same layer: pooling and the
+    mask in full, attention on `rows_sample` seeded (head, query block) rows, extrapolated
+    to the layer's rows."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    w = inp.workload
+    cu = inp.cu_seqlens.tolist()
+    q, k, v = inp.codes_f32("q"), inp.codes_f32("k"), inp.codes_f32("v")
+    qs, ks, vs = inp.scale_f64("q"), inp.scale_f64("k"), inp.scale_f64("v")
+    scale = 1.0 / math.sqrt(w.d)
+    t0 = time.perf_counter()
+    qp = O.pool_blocks(q, w.block, cu, scale=qs)
+    kp = O.pool_blocks(k, w.block, cu, scale=ks)
+    sc = O.block_scores(qp, kp, cu, w.block, scale)
+    keeps = [O.block_keep(s, w.alpha) for s in sc]
+    t1 = time.perf_counter()
+    nb, off = O.request_blocks(cu, w.block)
+    rng = np.random.default_rng(seed)
+    rows = [(int(rng.integers(w.Hq)), int(rng.integers(off[-1]))) for _ in range(rows_sample)]
+    O.masked_causal_attention(q, k, v, keeps, cu, w.block, scale, rows=rows, q_scale=qs,
+                              k_scale=ks, v_scale=vs)
+    t2 = time.perf_counter()
+    total_rows = w.Hq * off[-1]
+    ms = 1e3 * ((t1 - t0) + (t2 - t1) * total_rows / rows_sample)
+    sample = (f"pool+mask in full ({1e3 * (t1 - t0):.0f} ms) + attention on {rows_sample} of "
+              f"{total_rows} (head, query-block) rows ({1e3 * (t2 - t1):.0f} ms), "
+              f"extrapolated to the layer")
+    return {"value": round(ms, 3), "unit": "ms/layer", "cores": cores, "kind": "oracle",
+            "sample": sample}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl" if args.impl == "native" else "gloo",
+            timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = S.WORKLOADS[args.workload]
+    inp = S.make_inputs(args.workload)
+    times = []
+    cb = None
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        cb = cpu_baseline(inp, rows_sample=args.ref_rows, seed=5 + i)
+        if i >= args.warmup:
+            times.append(cb["value"])
+    v = statistics.median(times)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms/layer",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": v, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, args), "cpu_baseline": dict(cb, value=v),
+            "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(w, args):
+    return {"workload": f"{w.name}: L={'+'.join(map(str, w.seqlens)) if len(w.seqlens) < 9 else w.total_tokens} "
+                        f"Hq={w.Hq} Hkv={w.Hkv} d={w.d} block={w.block} alpha={w.alpha} "
+                        f"{w.dtype}" + (f" paged{w.page_size}" if w.page_size else ""),
+            "tokens": w.total_tokens, "requests": w.batch, "parallelism": f"replicas{args.gpus}",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
+def run_native(args, world, rank, local):
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = S.WORKLOADS[args.workload]
+    inp = S.make_inputs(args.workload, seed=S.DEFAULT_SEEDS[w.name] + 1000 * rank)
+    layer = Layer(inp, dev)
+    peaks, peak_src = _peaks()
+
+    for _ in range(args.warmup):
+        layer.step()
+    torch.cuda.synchronize(dev)
+    fp.check_status(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = Clocks(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        out, cnt, idx = layer.step(evs[i])
+    t_end.record()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    fp.check_status(dev)
+    total_ms = t_start.elapsed_time(t_end)
+    ms_step = max_over_ranks(total_ms / args.steps, world, dev)
+    pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    mask_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    alg, executed, density = work_counts(w, cnt, idx, layer.batch)
+    pm_bytes = pool_mask_bytes(w)
+    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    if w.dtype == "e4m3":
+        peak_t *= 2.0   # e4m3 dense rate = 2x bf16 (nominal ratio); no measured e4m3 peak
+    traffic = None
+    tf = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if os.path.exists(tf):
+        t = json.load(open(tf)).get(w.name)
+        if t:
+            traffic = t
+    roof = {"bound": "tensor", "achieved": round(alg / (attn_ms * 1e-3) / 1e12, 2),
+            "peak": peak_t, "unit": "TFLOP/s",
+            "frac": round(alg / (attn_ms * 1e-3) / 1e12 / peak_t, 4), "traffic": traffic,
+            "peak_source": f"{peak_src} bf16 sustained" + (" x2 (e4m3 nominal ratio)"
+                                                          if w.dtype == "e4m3" else ""),
+            "executed_tflops": round(executed / (attn_ms * 1e-3) / 1e12, 2),
+            "executed_frac": round(executed / (attn_ms * 1e-3) / 1e12 / peak_t, 4)}
+
+    # e2e: host (pinned) inputs -> device, the layer, output -> host, per step
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(layer, inp, dev, args, world)
+
+    if rank == 0:
+        cb = None
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline(inp, rows_sample=args.ref_rows)
+        line = {
+            "metric": METRIC, "value": round(ms_step / world, 4), "unit": "ms/layer",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": _config(w, args),
+            "stages_ms": {"pool": round(pool_ms, 4), "mask": round(mask_ms, 4),
+                          "attn": round(attn_ms, 4)},
+            "pool_mask": {"bytes": pm_bytes,
+                          "gbs": round(pm_bytes / ((pool_ms + mask_ms) * 1e-3) / 1e9, 1),
+                          "frac_hbm": round(pm_bytes / ((pool_ms + mask_ms) * 1e-3) / 1e9 /
+                                            peaks["hbm_gbs"], 4),
+                          "pool_frac_hbm": round(pm_bytes / (pool_ms * 1e-3) / 1e9 /
+                                                 peaks["hbm_gbs"], 4)},
+            "block_density": round(density, 5),
+            "attn_tflop": {"algorithmic": round(alg / 1e12, 3),
+                           "executed": round(executed / 1e12, 3)},
+            "roofline": roof,
+            "cpu_baseline": cb,
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(layer, inp, dev, args, world):
+    """Same metric through the public API with host buffers: every step copies Q, K, V from
+    pinned host memory, runs the layer, and copies the output back."""
+    hq = inp.q.pin_memory()
+    hk = (inp.k_cache if inp.k_cache is not None else inp.k).pin_memory()
+    hv = (inp.v_cache if inp.v_cache is not None else inp.v).pin_memory()
+    hout = torch.empty(layer.q.shape, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv = torch.empty_like(hq, device=dev), torch.empty_like(hk, device=dev), \
+        torch.empty_like(hv, device=dev)
+    saved = (layer.q, layer.k, layer.v, layer.paged)
+    layer.q = dq
+    if layer.paged is not None:
+        layer.paged = fp.PagedKV(dk, dv, layer.paged.page_table)
+    else:
+        layer.k, layer.v = dk, dv
+    steps = max(1, min(args.steps, 5))
+
+    def one():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        out, _, _ = layer.step()
+        hout.copy_(out, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+    layer.q, layer.k, layer.v, layer.paged = saved
+    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + \
+        hv.numel() * hv.element_size()
+    return {"value": round(ms / world, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": hout.numel() * hout.element_size(), "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="llama128k", choices=sorted(S.WORKLOADS))
+    ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_native(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

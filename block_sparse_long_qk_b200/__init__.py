@@ -1,0 +1,303 @@
+"""Block-sparse causal prefill attention for B200 (FlashPrefill-style), Python binding.
+
+Thin ctypes layer over ``libfpsparse.so`` (declared in ``include/fpsparse.h``). It only
+marshals arguments: torch is used for device memory and streams, and every step of the
+path runs in the library's CUDA kernels. There is no CPU fallback: if the library is
+missing or fails to load, every call raises.
+
+The path (names follow "FlashPrefill: Instantaneous Pattern Discovery and Thresholding for
+Ultra-Fast Long-Context Prefilling", technical summary section 2):
+
+    q_pool, k_pool     = pool_qk(q, k, block)                      # 2.A block means
+    mask, kv_cnt, kv_idx = build_block_mask(q_pool, k_pool, alpha)   # 2.B max-based threshold
+    out, lse           = sparse_prefill_attn(q, k, v, kv_cnt, kv_idx)  # 2.C physical skip
+
+``sparse_prefill`` runs all three. Paged K/V (``PagedKV``) and varlen batches (``Batch``)
+follow "FlashPrefill V2: Block-Sparse Prefill Attention for Long-Context LLM Serving",
+Abstract (paged KV cache, continuous batching).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+import re
+
+import torch
+
+__all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_attn",
+           "sparse_prefill_attn_paged", "sparse_prefill", "check_status", "workspace",
+           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "header_symbols"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfpsparse.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "fpsparse.h")
+
+FP_OK = 0
+FP_DTYPE_BF16, FP_DTYPE_E4M3 = 0, 1
+FORCE_FIRST, FORCE_DIAG = 1, 2
+_ERRORS = {-1: "FP_ERR_INVALID_ARG", -2: "FP_ERR_UNSUPPORTED", -3: "FP_ERR_CUDA",
+           -4: "FP_ERR_TIMEOUT", -5: "FP_ERR_BAD_INDEX"}
+
+_p, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_SIGNATURES = {
+    "fp_version": (_i, []),
+    "fp_last_error_string": (ctypes.c_char_p, []),
+    "fp_workspace_size": (_sz, []),
+    "fp_pool_qk": (_i, [_p, _p, _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i,
+                        _i, _p, _p, _p]),
+    "fp_build_block_mask": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _f, _i, _p, _p, _p,
+                                 _p]),
+    "fp_sparse_prefill_attn": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i,
+                                    _i, _i, _i, _f, _p, _p, _p, _p, _p, _p]),
+    "fp_sparse_prefill_attn_paged": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _i, _i, _i, _i,
+                                          _i, _i, _i, _i, _p, _i, _i, _i, _f, _p, _p, _p, _p,
+                                          _p, _p]),
+    "fp_check_status": (_i, [_p, _p]),
+}
+
+
+class FpError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{_ERRORS.get(code, code)}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def library():
+    """The loaded C library. Raises if it is missing (build it with
+    ``python -m block_sparse_long_qk_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise FpError(-3, f"{LIB_PATH} not found; build it with "
+                              "`python -m block_sparse_long_qk_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def header_symbols():
+    """Names of the functions declared in include/fpsparse.h."""
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(fp_\w+)\s*\(", txt,
+                                 flags=re.M)))
+
+
+def _check(rc):
+    if rc != FP_OK:
+        raise FpError(rc, library().fp_last_error_string().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return FP_DTYPE_BF16
+    if t.dtype == torch.float8_e4m3fn:
+        return FP_DTYPE_E4M3
+    raise TypeError(f"unsupported storage dtype {t.dtype} (bf16 or float8_e4m3fn)")
+
+
+@dataclasses.dataclass
+class Batch:
+    """A varlen batch: host lengths plus the device index arrays the kernels read."""
+    seqlens: tuple
+    block: int
+    cu_seqlens: torch.Tensor    # int32 [B+1] on the device
+    cu_blocks: torch.Tensor     # int32 [B+1] on the device
+    total_tokens: int
+    total_blocks: int
+    max_blocks: int
+
+    @staticmethod
+    def make(seqlens, block, device):
+        seqlens = tuple(int(s) for s in seqlens)
+        nb = [(s + block - 1) // block for s in seqlens]
+        cu = [0]
+        for s in seqlens:
+            cu.append(cu[-1] + s)
+        cb = [0]
+        for n in nb:
+            cb.append(cb[-1] + n)
+        return Batch(seqlens, block, torch.tensor(cu, dtype=torch.int32, device=device),
+                     torch.tensor(cb, dtype=torch.int32, device=device), cu[-1], cb[-1],
+                     max(nb) if nb else 0)
+
+    @property
+    def size(self):
+        return len(self.seqlens)
+
+    def _ptrs(self):
+        if self.size == 1:
+            return None, None
+        return _ptr(self.cu_seqlens), _ptr(self.cu_blocks)
+
+
+@dataclasses.dataclass
+class PagedKV:
+    """K/V caches [num_pages, page_size, Hkv, d] and the int32 page table [B, max_pages]."""
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    page_table: torch.Tensor
+
+    @property
+    def page_size(self):
+        return self.k_cache.shape[1]
+
+
+_workspaces = {}
+
+
+def workspace(device):
+    """A zeroed per-device status workspace (allocated once by torch)."""
+    device = torch.device(device)
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(key)
+    if ws is None:
+        n = library().fp_workspace_size()
+        ws = torch.zeros(max(256, n), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def check_status(device=None, ws=None):
+    """Waits for the current stream and raises if an attention launch recorded a pipeline
+    timeout or an out-of-range index since the last check."""
+    if ws is None:
+        ws = workspace(device if device is not None else torch.device("cuda"))
+    _check(library().fp_check_status(_ptr(ws), _stream(ws.device)))
+
+
+def _batch_for(q, block, batch):
+    if batch is None:
+        return Batch.make((q.shape[0],), block, q.device)
+    if batch.block != block:
+        raise ValueError("batch was built for a different block size")
+    return batch
+
+
+def pool_qk(q, k, block=128, *, batch: Batch | None = None, q_scale=None, k_scale=None,
+            paged: PagedKV | None = None):
+    """Block means of Q [T,Hq,d] and K [T,Hkv,d] (or the paged K cache) -> float32
+    q_pool [Hq, nblk, d], k_pool [Hkv, nblk, d]."""
+    T, Hq, d = q.shape
+    kk = paged.k_cache if paged is not None else k
+    Hkv = kk.shape[-2]
+    b = _batch_for(q, block, batch)
+    q_pool = torch.empty((Hq, b.total_blocks, d), dtype=torch.float32, device=q.device)
+    k_pool = torch.empty((Hkv, b.total_blocks, d), dtype=torch.float32, device=q.device)
+    cu, cb = b._ptrs()
+    if paged is not None and cu is None:
+        cu, cb = _ptr(b.cu_seqlens), _ptr(b.cu_blocks)
+    pt = paged.page_table if paged is not None else None
+    _check(library().fp_pool_qk(
+        _ptr(q), _ptr(kk), _dtype_code(q), _ptr(q_scale), _ptr(k_scale), cu, cb, b.size, T,
+        b.total_blocks, Hq, Hkv, d, block, _ptr(pt), paged.page_size if paged else 0,
+        pt.shape[1] if pt is not None else 0, kk.shape[0] if pt is not None else 0,
+        _ptr(q_pool), _ptr(k_pool), _stream(q.device)))
+    return q_pool, k_pool
+
+
+def build_block_mask(q_pool, k_pool, alpha=0.1, *, block=128, batch: Batch | None = None,
+                     scale=None, flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True):
+    """Max-based dynamic threshold on the pooled block scores -> (mask_bits or None
+    [Hq, nblk, words] uint32 viewed as int32, kv_cnt [Hq, nblk] int32, kv_idx
+    [Hq, nblk, max_blocks] int32)."""
+    Hq, nblk, d = q_pool.shape
+    Hkv = k_pool.shape[0]
+    if batch is None:
+        batch = Batch.make((nblk * block,), block, q_pool.device)
+        batch = dataclasses.replace(batch, total_blocks=nblk, max_blocks=nblk)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    words = (batch.max_blocks + 31) // 32
+    dev = q_pool.device
+    bits = torch.zeros((Hq, nblk, words), dtype=torch.int32, device=dev) if mask_bits else None
+    kv_cnt = torch.empty((Hq, nblk), dtype=torch.int32, device=dev)
+    kv_idx = torch.empty((Hq, nblk, batch.max_blocks), dtype=torch.int32, device=dev)
+    cb = _ptr(batch.cu_blocks) if batch.size > 1 else None
+    _check(library().fp_build_block_mask(
+        _ptr(q_pool), _ptr(k_pool), cb, batch.size, nblk, batch.max_blocks, Hq, Hkv, d,
+        float(alpha), float(scale), int(flags), _ptr(bits), _ptr(kv_cnt), _ptr(kv_idx),
+        _stream(dev)))
+    return bits, kv_cnt, kv_idx
+
+
+def sparse_prefill_attn(q, k, v, kv_cnt, kv_idx, block=128, *, batch: Batch | None = None,
+                        scale=None, q_scale=None, k_scale=None, v_scale=None,
+                        return_lse=False, out=None, ws=None):
+    """Causal attention over the kept KV blocks -> (out bf16 [T,Hq,d], lse [Hq,T] or None)."""
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    b = _batch_for(q, block, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if return_lse else None
+    ws = workspace(q.device) if ws is None else ws
+    cu, cb = b._ptrs()
+    _check(library().fp_sparse_prefill_attn(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+        cu, cb, b.size, T, b.total_blocks, b.max_blocks, Hq, Hkv, d, block, float(scale),
+        _ptr(kv_cnt), _ptr(kv_idx), _ptr(out), _ptr(lse), _ptr(ws), _stream(q.device)))
+    return out, lse
+
+
+def sparse_prefill_attn_paged(q, paged: PagedKV, kv_cnt, kv_idx, batch: Batch, *,
+                              scale=None, q_scale=None, k_scale=None, v_scale=None,
+                              return_lse=False, out=None, ws=None):
+    """Same as ``sparse_prefill_attn`` with K/V read through the page table."""
+    T, Hq, d = q.shape
+    Hkv = paged.k_cache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if return_lse else None
+    ws = workspace(q.device) if ws is None else ws
+    pt = paged.page_table
+    _check(library().fp_sparse_prefill_attn_paged(
+        _ptr(q), _ptr(paged.k_cache), _ptr(paged.v_cache), _dtype_code(q), _ptr(q_scale),
+        _ptr(k_scale), _ptr(v_scale), _ptr(batch.cu_seqlens), _ptr(batch.cu_blocks),
+        batch.size, T, batch.total_blocks, batch.max_blocks, Hq, Hkv, d, batch.block, _ptr(pt),
+        paged.page_size, pt.shape[1], paged.k_cache.shape[0], float(scale), _ptr(kv_cnt),
+        _ptr(kv_idx), _ptr(out), _ptr(lse), _ptr(ws), _stream(q.device)))
+    return out, lse
+
+
+def sparse_prefill(q, k=None, v=None, alpha=0.1, block=128, *, batch: Batch | None = None,
+                   paged: PagedKV | None = None, scale=None, q_scale=None, k_scale=None,
+                   v_scale=None, return_lse=False, flags=FORCE_FIRST | FORCE_DIAG):
+    """The whole path: pool -> threshold/mask -> sparse attention. Returns
+    (out, lse or None, kv_cnt, kv_idx)."""
+    b = _batch_for(q, block, batch)
+    d = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    q_pool, k_pool = pool_qk(q, k, block, batch=b, q_scale=q_scale, k_scale=k_scale, paged=paged)
+    _, kv_cnt, kv_idx = build_block_mask(q_pool, k_pool, alpha, block=block, batch=b,
+                                         scale=scale, flags=flags, mask_bits=False)
+    if paged is not None:
+        out, lse = sparse_prefill_attn_paged(q, paged, kv_cnt, kv_idx, b, scale=scale,
+                                             q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,
+                                             return_lse=return_lse)
+    else:
+        out, lse = sparse_prefill_attn(q, k, v, kv_cnt, kv_idx, block, batch=b, scale=scale,
+                                       q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,
+                                       return_lse=return_lse)
+    return out, lse, kv_cnt, kv_idx

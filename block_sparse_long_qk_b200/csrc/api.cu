@@ -1,0 +1,281 @@
+// extern "C" entry points of libfpsparse.so: argument checks, then one kernel launch each.
+// Declarations and the contract of every call are in include/fpsparse.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "fp_common.cuh"
+#include "fp_launch.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared checks of the varlen description and head layout.
+int check_common(int dtype, const float* qs, const float* ks, const float* vs, bool need_v,
+                 const int32_t* cu_seqlens, const int32_t* cu_blocks, int batch,
+                 int total_tokens, int total_blocks, int Hq, int Hkv, int d, int block) {
+  if (dtype != FP_DTYPE_BF16 && dtype != FP_DTYPE_E4M3)
+    return fail(FP_ERR_INVALID_ARG, "dtype %d is neither FP_DTYPE_BF16 nor FP_DTYPE_E4M3", dtype);
+  if (dtype == FP_DTYPE_BF16 && (qs || ks || vs))
+    return fail(FP_ERR_INVALID_ARG, "bf16 inputs take no scales (pass NULL)");
+  if (dtype == FP_DTYPE_E4M3 && (!qs || !ks || (need_v && !vs)))
+    return fail(FP_ERR_INVALID_ARG, "e4m3 inputs need per-head scales");
+  if (d != 64 && d != 128) return fail(FP_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (block != 64 && block != 128)
+    return fail(FP_ERR_UNSUPPORTED, "block %d (supported: 64, 128)", block);
+  if (batch < 1) return fail(FP_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", batch);
+  if (batch > 1 && (!cu_seqlens || !cu_blocks))
+    return fail(FP_ERR_INVALID_ARG, "batch > 1 needs cu_seqlens and cu_blocks");
+  if ((cu_seqlens == nullptr) != (cu_blocks == nullptr))
+    return fail(FP_ERR_INVALID_ARG, "cu_seqlens and cu_blocks are both given or both NULL");
+  if (total_tokens < 0 || total_blocks < 0)
+    return fail(FP_ERR_INVALID_ARG, "negative token or block count");
+  if (cu_blocks == nullptr && total_blocks != (total_tokens + block - 1) / block)
+    return fail(FP_ERR_INVALID_ARG, "total_blocks %d != ceil(T / block) for one sequence",
+                total_blocks);
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+    return fail(FP_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq, Hkv);
+  return FP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp_version(void) { return 100; }
+
+const char* fp_last_error_string(void) { return g_err.c_str(); }
+
+size_t fp_workspace_size(void) { return 256; }
+
+int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
+               const float* k_scale, const int32_t* cu_seqlens, const int32_t* cu_blocks,
+               int batch, int total_tokens, int total_blocks, int Hq, int Hkv, int d,
+               int block, const int32_t* k_page_table, int page_size, int max_pages,
+               int num_pages, float* q_pool, float* k_pool, void* stream) {
+  g_err.clear();
+  int rc = check_common(dtype, q_scale, k_scale, nullptr, false, cu_seqlens, cu_blocks, batch,
+                        total_tokens, total_blocks, Hq, Hkv, d, block);
+  if (rc) return rc;
+  if (!q || !k || !q_pool || !k_pool) return fail(FP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool))
+    return fail(FP_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (k_page_table) {
+    if (page_size < 16 || page_size % 16 || block % page_size || max_pages < 1 || num_pages < 1)
+      return fail(FP_ERR_INVALID_ARG, "page_size %d must be a multiple of 16 dividing block %d",
+                  page_size, block);
+    if (cu_blocks == nullptr)
+      return fail(FP_ERR_INVALID_ARG, "a paged K needs cu_seqlens/cu_blocks");
+  }
+  if (total_blocks == 0) return FP_OK;
+  fp::PoolArgs a{};
+  a.num_pages = num_pages;
+  a.q = static_cast<const uint8_t*>(q);
+  a.k = static_cast<const uint8_t*>(k);
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.cu_seqlens = cu_seqlens;
+  a.cu_blocks = cu_blocks;
+  a.page_table = k_page_table;
+  a.q_pool = q_pool;
+  a.k_pool = k_pool;
+  a.batch = batch;
+  a.total_tokens = total_tokens;
+  a.total_blocks = total_blocks;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.block = block;
+  a.page_size = page_size;
+  a.max_pages = max_pages;
+  cudaError_t e = fp::launch_pool(a, dtype == FP_DTYPE_E4M3, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP_OK : cuda_fail(e, "pool kernel launch");
+}
+
+int fp_build_block_mask(const float* q_pool, const float* k_pool, const int32_t* cu_blocks,
+                        int batch, int total_blocks, int max_blocks, int Hq, int Hkv, int d,
+                        float alpha, float scale, int flags, uint32_t* mask_bits,
+                        int32_t* kv_cnt, int32_t* kv_idx, void* stream) {
+  g_err.clear();
+  if (!q_pool || !k_pool || !kv_cnt || !kv_idx) return fail(FP_ERR_INVALID_ARG, "null pointer");
+  if (batch < 1 || (batch > 1 && !cu_blocks))
+    return fail(FP_ERR_INVALID_ARG, "batch > 1 needs cu_blocks");
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv)
+    return fail(FP_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq, Hkv);
+  if (d != 64 && d != 128) return fail(FP_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (!(alpha >= 0.f && alpha <= 1.f)) return fail(FP_ERR_INVALID_ARG, "alpha must be in [0, 1]");
+  if (total_blocks < 0 || max_blocks < 0 || (total_blocks > 0 && max_blocks < 1))
+    return fail(FP_ERR_INVALID_ARG, "bad block counts");
+  if (cu_blocks == nullptr && max_blocks != total_blocks)
+    return fail(FP_ERR_INVALID_ARG, "one sequence: max_blocks must equal total_blocks");
+  if (!aligned16(q_pool) || !aligned16(k_pool))
+    return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
+  if (total_blocks == 0) return FP_OK;
+  const int G = Hq / Hkv;
+  const int nb = fp::mask_blocks_per_cta(G, d, max_blocks);
+  if (nb == 0)
+    return fail(FP_ERR_UNSUPPORTED, "%d blocks per request with %d heads per KV head exceed the "
+                "shared-memory score rows of the mask kernel", max_blocks, G);
+  fp::MaskArgs a{};
+  a.q_pool = q_pool;
+  a.k_pool = k_pool;
+  a.cu_blocks = cu_blocks;
+  a.mask_bits = mask_bits;
+  a.kv_cnt = kv_cnt;
+  a.kv_idx = kv_idx;
+  a.batch = batch;
+  a.total_blocks = total_blocks;
+  a.max_blocks = max_blocks;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.G = G;
+  a.NB = nb;
+  a.log_alpha = alpha > 0.f ? logf(alpha) : -INFINITY;
+  a.scale = scale;
+  a.flags = flags;
+  cudaError_t e = fp::launch_mask(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP_OK : cuda_fail(e, "mask kernel launch");
+}
+
+static int attn_common(const void* q, const void* k, const void* v, int dtype,
+                       const float* q_scale, const float* k_scale, const float* v_scale,
+                       const int32_t* cu_seqlens, const int32_t* cu_blocks, int batch,
+                       int total_tokens, int total_blocks, int max_blocks, int Hq, int Hkv,
+                       int d, int block, const int32_t* page_table, int page_size,
+                       int max_pages, int num_pages, float scale, const int32_t* kv_cnt,
+                       const int32_t* kv_idx, void* out, float* lse, void* workspace,
+                       void* stream) {
+  g_err.clear();
+  int rc = check_common(dtype, q_scale, k_scale, v_scale, true, cu_seqlens, cu_blocks, batch,
+                        total_tokens, total_blocks, Hq, Hkv, d, block);
+  if (rc) return rc;
+  if (!q || !k || !v || !out || !kv_cnt || !kv_idx || !workspace)
+    return fail(FP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(FP_ERR_INVALID_ARG, "Q, K, V and out must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (dtype == FP_DTYPE_E4M3 && !(d == 128 && block == 128))
+    return fail(FP_ERR_UNSUPPORTED, "e4m3 attention supports d = 128, block = 128");
+  if (cu_blocks == nullptr && max_blocks != total_blocks)
+    return fail(FP_ERR_INVALID_ARG, "one sequence: max_blocks must equal total_blocks");
+  if (page_table) {
+    if (page_size < 16 || page_size % 16 || block % page_size || max_pages < 1 || num_pages < 1)
+      return fail(FP_ERR_INVALID_ARG, "page_size %d must be a multiple of 16 dividing block %d",
+                  page_size, block);
+    if (cu_blocks == nullptr)
+      return fail(FP_ERR_INVALID_ARG, "paged attention needs cu_seqlens/cu_blocks");
+  }
+  const int G = Hq / Hkv;
+  fp::AttnArgs a{};
+  a.cu_seqlens = cu_seqlens;
+  a.cu_blocks = cu_blocks;
+  a.kv_cnt = kv_cnt;
+  a.kv_idx = kv_idx;
+  a.page_table = page_table;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.status = static_cast<uint32_t*>(workspace);
+  a.batch = batch;
+  a.total_tokens = total_tokens;
+  a.total_blocks = total_blocks;
+  a.max_blocks = max_blocks;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.block = block;
+  a.page_size = page_size;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  a.pair_heads = (G % 2 == 0) ? 1 : 0;
+  a.num_items = a.pair_heads ? (Hq / 2) * total_blocks : Hq * total_blocks;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  fp::AttnLaunch L{};
+  L.q = q;
+  L.k = k;
+  L.v = v;
+  L.e4m3 = dtype == FP_DTYPE_E4M3;
+  L.paged = page_table != nullptr;
+  L.d = d;
+  L.kv_rows = page_table ? static_cast<long long>(num_pages) * page_size : total_tokens;
+  L.seg_rows = page_table ? page_size : block;
+  if (total_blocks == 0) return FP_OK;
+  cudaError_t e = fp::launch_attn(a, L, block, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return fail(FP_ERR_UNSUPPORTED, "unsupported d/block/dtype");
+  return e == cudaSuccess ? FP_OK : cuda_fail(e, "attention kernel launch");
+}
+
+int fp_sparse_prefill_attn(const void* q, const void* k, const void* v, int dtype,
+                           const float* q_scale, const float* k_scale, const float* v_scale,
+                           const int32_t* cu_seqlens, const int32_t* cu_blocks, int batch,
+                           int total_tokens, int total_blocks, int max_blocks, int Hq,
+                           int Hkv, int d, int block, float scale, const int32_t* kv_cnt,
+                           const int32_t* kv_idx, void* out, float* lse, void* workspace,
+                           void* stream) {
+  return attn_common(q, k, v, dtype, q_scale, k_scale, v_scale, cu_seqlens, cu_blocks, batch,
+                     total_tokens, total_blocks, max_blocks, Hq, Hkv, d, block, nullptr, 0, 0,
+                     0, scale, kv_cnt, kv_idx, out, lse, workspace, stream);
+}
+
+int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void* v_cache,
+                                 int dtype, const float* q_scale, const float* k_scale,
+                                 const float* v_scale, const int32_t* cu_seqlens,
+                                 const int32_t* cu_blocks, int batch, int total_tokens,
+                                 int total_blocks, int max_blocks, int Hq, int Hkv, int d,
+                                 int block, const int32_t* page_table, int page_size,
+                                 int max_pages, int num_pages, float scale,
+                                 const int32_t* kv_cnt, const int32_t* kv_idx, void* out,
+                                 float* lse, void* workspace, void* stream) {
+  if (!page_table) {
+    g_err = "paged attention needs a page table";
+    return FP_ERR_INVALID_ARG;
+  }
+  return attn_common(q, k_cache, v_cache, dtype, q_scale, k_scale, v_scale, cu_seqlens,
+                     cu_blocks, batch, total_tokens, total_blocks, max_blocks, Hq, Hkv, d,
+                     block, page_table, page_size, max_pages, num_pages, scale, kv_cnt, kv_idx,
+                     out, lse, workspace, stream);
+}
+
+int fp_check_status(void* workspace, void* stream) {
+  g_err.clear();
+  if (!workspace) return fail(FP_ERR_INVALID_ARG, "null workspace");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  if (word != 0) {
+    e = cudaMemsetAsync(workspace, 0, sizeof(word), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  }
+  if (word & fp::kStatusTimeout)
+    return fail(FP_ERR_TIMEOUT, "a pipeline wait in the attention kernel timed out");
+  if (word & fp::kStatusBadIndex)
+    return fail(FP_ERR_BAD_INDEX, "an index list or page table entry was out of range");
+  return FP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,531 @@
+// Stage 3: block-sparse causal attention over the kept KV blocks (contiguous and paged KV).
+//
+// "FlashPrefill: Instantaneous Pattern Discovery and Thresholding for Ultra-Fast Long-Context
+// Prefilling", technical summary 2.C: masked blocks are skipped physically -- the kernel walks
+// the index list of kept blocks and points its loads straight at them, running no control
+// logic for the blocks in between. "FlashPrefill V2: Block-Sparse Prefill Attention for
+// Long-Context LLM Serving", Abstract: query heads that share a KV head are packed onto the
+// same K/V loads (PackGQA), FP8 inputs, paged KV cache and continuous batching.
+//
+// B200 design (one CTA = two 128-row query tiles that read the same KV head):
+//   warp 0      TMA producer: both Q tiles once, then K and V tiles of the union of the two
+//               tiles' kept-block lists into a 2-deep K ring and a 2-deep V ring.
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer. Per union block it issues
+//               S_t = Q_t K^T for each tile t that kept the block, and, before that, the
+//               pending O_t += P_t V of the tile's previous block. The two tiles therefore
+//               alternate on the tensor core while the other tile's softmax runs (the sm_100
+//               counterpart of the pages' pingpong schedule).
+//   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread per query row reads
+//               its S row from TMEM, applies the causal mask on the diagonal block, keeps a
+//               running max with lazy rescaling of O (only when the max grows by more than
+//               2^8), writes P (bf16 or e4m3) back into the S columns of TMEM, and finally
+//               normalises O and writes the bf16 output row (plus the row's log-sum-exp).
+// TMEM: S0 | S1 | O0 | O1 (fp32 accumulators, 128 lanes); P_t aliases the first columns of S_t
+// and is consumed by the PV MMA straight from TMEM. All waits are bounded (fp_common.cuh).
+#include <math.h>
+
+#include "fp_common.cuh"
+#include "fp_launch.h"
+
+namespace fp {
+
+template <int D, int BN, bool FP8>
+struct AttnCfg {
+  static constexpr int kBM = 128;
+  static constexpr int kEB = FP8 ? 1 : 2;
+  static constexpr int kChunkEl = 128 / kEB;         // elements per 128-byte swizzle row
+  static constexpr int kNChunk = D / kChunkEl;
+  static constexpr int kQBytes = kBM * D * kEB;
+  static constexpr int kKVBytes = BN * D * kEB;
+  static constexpr int kKSt = 2, kVSt = 2;
+  static constexpr int kKStep = FP8 ? 32 : 16;       // MMA K per instruction
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kQBytes;
+  static constexpr int kVOff = kKOff + kKSt * kKVBytes;
+  static constexpr int kBarOff = kVOff + kVSt * kKVBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+  static constexpr int kTmemUsed = 2 * BN + 2 * D;          // S0 S1 O0 O1
+  static constexpr int kTmemCols = kTmemUsed <= 256 ? 256 : 512;  // power-of-2 allocation
+  static constexpr uint32_t kS0 = 0, kS1 = BN, kO0 = 2 * BN, kO1 = 2 * BN + D;
+  static constexpr int kThreads = 384;
+  static_assert(kTmemUsed <= 512, "S and O tiles of both query tiles must fit in TMEM");
+};
+
+struct Tile {
+  int h, Ig, I, q_lo, nvalid, cnt;  // nvalid = 0 marks an absent tile
+  const int32_t* list;
+};
+
+struct Shared {  // placed at kBarOff
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full[2], p_full[2], o_final[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+
+// Next entry of a kept-block list that is a valid causal block index (0 <= J <= I), or -1.
+// Invalid entries are skipped; `report` records them once in the status word.
+__device__ __forceinline__ int next_valid(const int32_t* list, int cnt, int& i, int I,
+                                          uint32_t* status, bool report) {
+  while (i < cnt) {
+    const int J = __ldg(list + i);
+    ++i;
+    if (J >= 0 && J <= I) return J;
+    if (report) record_status(status, kStatusBadIndex);
+  }
+  return -1;
+}
+
+// Walks the ascending union of two kept-block lists; `bits` says which tiles kept the block.
+struct UnionWalk {
+  const int32_t *l0, *l1;
+  int c0, c1, i0, i1, I0, I1, a, b;
+  __device__ void init(const Tile& t0, const Tile& t1) {
+    l0 = t0.list; l1 = t1.list; c0 = t0.cnt; c1 = t1.cnt; I0 = t0.I; I1 = t1.I;
+    i0 = i1 = 0;
+    a = next_valid(l0, c0, i0, I0, nullptr, false);
+    b = next_valid(l1, c1, i1, I1, nullptr, false);
+  }
+  __device__ bool next(int& J, int& bits) {
+    if (a < 0 && b < 0) return false;
+    if (b < 0 || (a >= 0 && a < b)) { J = a; bits = 1; a = next_valid(l0, c0, i0, I0, nullptr, false); }
+    else if (a < 0 || b < a) { J = b; bits = 2; b = next_valid(l1, c1, i1, I1, nullptr, false); }
+    else { J = a; bits = 3; a = next_valid(l0, c0, i0, I0, nullptr, false); b = next_valid(l1, c1, i1, I1, nullptr, false); }
+    return true;
+  }
+};
+
+__device__ __forceinline__ void request_of(const AttnArgs& a, int Ig, int& b, int& base,
+                                           int& len, int& blk0) {
+  if (a.cu_blocks == nullptr) { b = 0; base = 0; len = a.total_tokens; blk0 = 0; return; }
+  b = find_request(a.cu_blocks, a.batch, Ig);
+  base = __ldg(a.cu_seqlens + b);
+  len = __ldg(a.cu_seqlens + b + 1) - base;
+  blk0 = __ldg(a.cu_blocks + b);
+}
+
+// Work item -> two tiles sharing one KV head. Items run heaviest-first (late query blocks
+// have the longest causal rows).
+__device__ __forceinline__ void make_tiles(const AttnArgs& a, int item, Tile* t, int& g,
+                                           int& b, int& base, int& len) {
+  int blk0;
+  if (a.pair_heads) {
+    const int npairs = a.Hq / 2;
+    const int Ig = a.total_blocks - 1 - item / npairs;
+    const int p = item % npairs;
+    request_of(a, Ig, b, base, len, blk0);
+    for (int s = 0; s < 2; ++s) { t[s].h = 2 * p + s; t[s].Ig = Ig; }
+  } else {
+    // Query heads do not pair up on a KV head (odd group size): one tile per CTA.
+    const int Ig = a.total_blocks - 1 - item / a.Hq;
+    const int h = item % a.Hq;
+    request_of(a, Ig, b, base, len, blk0);
+    t[0].h = h; t[0].Ig = Ig;
+    t[1].h = h; t[1].Ig = -1;
+  }
+  g = t[0].h / (a.Hq / a.Hkv);
+  for (int s = 0; s < 2; ++s) {
+    if (t[s].Ig < 0) { t[s].nvalid = 0; t[s].cnt = 0; t[s].list = a.kv_idx; t[s].I = -1; t[s].q_lo = 0; continue; }
+    t[s].I = t[s].Ig - blk0;
+    t[s].q_lo = base + t[s].I * a.block;
+    t[s].nvalid = min(a.block, len - t[s].I * a.block);
+    const size_t row = static_cast<size_t>(t[s].h) * a.total_blocks + t[s].Ig;
+    t[s].cnt = __ldg(a.kv_cnt + row);
+    t[s].cnt = max(0, min(t[s].cnt, a.max_blocks));
+    t[s].list = a.kv_idx + row * a.max_blocks;
+  }
+}
+
+template <int D, int BN, bool FP8, bool PAGED>
+__global__ void __launch_bounds__(384, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  using C = AttnCfg<D, BN, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  // Swizzled TMA tiles and UMMA descriptors assume 1024-byte aligned shared addresses.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  Shared& sh = *reinterpret_cast<Shared*>(smem + C::kBarOff);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // A timeout recorded earlier in this workspace makes later CTAs exit at once, so one
+  // broken pipeline cannot hold the GPU for a 2 s wait per CTA. fp_check_status clears it.
+  if (threadIdx.x == 0)
+    sh.abort_flag = (a.status != nullptr && (*reinterpret_cast<volatile uint32_t*>(a.status) &
+                                             kStatusTimeout)) ? 1 : 0;
+  __syncthreads();
+  if (sh.abort_flag) return;
+
+  Tile tl[2];
+  int g, b, base, len;
+  make_tiles(a, blockIdx.x, tl, g, b, base, len);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sh.q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.k_full[i], 1); mbar_init(&sh.k_empty[i], 1);
+      mbar_init(&sh.v_full[i], 1); mbar_init(&sh.v_empty[i], 1);
+      mbar_init(&sh.s_full[i], 1); mbar_init(&sh.p_full[i], 128); mbar_init(&sh.o_final[i], 1);
+    }
+    mbar_init(&sh.drain, 1);
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&sh.tmem_base, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      const int ntiles = tl[1].nvalid > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(&sh.q_full, ntiles * C::kQBytes);
+      for (int s = 0; s < ntiles; ++s)
+        for (int c = 0; c < C::kNChunk; ++c)
+          tma_load_3d(smem + C::kQOff + s * C::kQBytes + c * (C::kBM * 128), &tm_q, &sh.q_full,
+                      c * C::kChunkEl, tl[s].h, tl[s].q_lo);
+      UnionWalk uw;
+      uw.init(tl[0], tl[1]);
+      int J, bits;
+      for (int k = 0; uw.next(J, bits); ++k) {
+        if (sh.abort_flag) break;
+        const int ks = k % C::kKSt, vs = k % C::kVSt;
+        // Row coordinates of the block's segments (whole block, or one per page).
+        constexpr int kSegRows = PAGED ? 0 : BN;
+        const int seg_rows = PAGED ? a.page_size : kSegRows;
+        const int nseg = BN / seg_rows;
+        for (int which = 0; which < 2; ++which) {
+          const int st = which == 0 ? ks : vs;
+          uint64_t* full = which == 0 ? &sh.k_full[st] : &sh.v_full[st];
+          uint64_t* empty = which == 0 ? &sh.k_empty[st] : &sh.v_empty[st];
+          const int use = k / (which == 0 ? C::kKSt : C::kVSt);
+          if (use > 0 && !mbar_wait(empty, (use - 1) & 1)) {
+            record_status(a.status, kStatusTimeout); sh.abort_flag = 1; break;
+          }
+          mbar_arrive_expect_tx(full, C::kKVBytes);
+          uint8_t* dst = smem + (which == 0 ? C::kKOff : C::kVOff) + st * C::kKVBytes;
+          const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;
+          for (int sgi = 0; sgi < nseg; ++sgi) {
+            int row;
+            const int tok = J * BN + sgi * seg_rows;  // request-local first token
+            if constexpr (PAGED) {
+              const int pages_req = (len + a.page_size - 1) / a.page_size;
+              const int lp = tok / a.page_size;
+              row = a.num_pages * a.page_size;  // past the end: TMA fills zeros
+              if (lp < pages_req && lp < a.max_pages) {
+                const int pid = __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp);
+                if (pid >= 0 && pid < a.num_pages) row = pid * a.page_size;
+                else record_status(a.status, kStatusBadIndex);
+              }
+            } else {
+              row = base + tok;
+            }
+            for (int c = 0; c < C::kNChunk; ++c)
+              tma_load_3d(dst + c * (BN * 128) + sgi * (seg_rows * 128), tm, full,
+                          c * C::kChunkEl, g, row);
+          }
+        }
+        if (sh.abort_flag) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = FP8 ? 0u : 1u;
+      constexpr uint32_t idesc_s = make_idesc(fmt, fmt, 0, 128, BN);
+      constexpr uint32_t idesc_o = make_idesc(fmt, fmt, 1, 128, D);
+      const uint32_t sbase = smem_u32(smem);
+      auto s_col = [](int t) -> uint32_t { return t == 0 ? C::kS0 : C::kS1; };
+      auto o_col = [](int t) -> uint32_t { return t == 0 ? C::kO0 : C::kO1; };
+      bool ok = mbar_wait(&sh.q_full, 0);
+      tc_fence_after();
+      int n[2] = {0, 0}, pend[2] = {-1, -1};
+      int vusers[2] = {0, 0};
+      auto issue_pv = [&](int t) -> bool {
+        const int k = pend[t];
+        const int vs = k % C::kVSt;
+        if (!mbar_wait(&sh.p_full[t], (n[t] - 1) & 1)) return false;
+        if (!mbar_wait(&sh.v_full[vs], (k / C::kVSt) & 1)) return false;
+        tc_fence_after();
+        const uint32_t vaddr = sbase + C::kVOff + vs * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < BN / C::kKStep; ++kk) {
+          const uint64_t bdesc = make_sdesc(vaddr + kk * (C::kKStep / 8) * 1024, BN * 128, 1024);
+          const uint32_t a_tm = tmem + s_col(t) + kk * 8;
+          const uint32_t acc = (n[t] > 1 || kk > 0) ? 1u : 0u;
+          if constexpr (FP8) mma_f8_ts(tmem + o_col(t), a_tm, bdesc, idesc_o, acc);
+          else mma_f16_ts(tmem + o_col(t), a_tm, bdesc, idesc_o, acc);
+        }
+        if (--vusers[vs] == 0) tc_commit(&sh.v_empty[vs]);
+        pend[t] = -1;
+        return true;
+      };
+      UnionWalk uw;
+      uw.init(tl[0], tl[1]);
+      int J, bits;
+      for (int k = 0; ok && uw.next(J, bits); ++k) {
+        if (sh.abort_flag) { ok = false; break; }
+        const int ks = k % C::kKSt;
+        if (!mbar_wait(&sh.k_full[ks], (k / C::kKSt) & 1)) { ok = false; break; }
+        tc_fence_after();
+        vusers[k % C::kVSt] = __popc(bits);
+        const uint32_t kaddr = sbase + C::kKOff + ks * C::kKVBytes;
+        // Tiles that kept this block: finish their previous block (PV), then S = Q K^T.
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!((bits >> t) & 1)) continue;
+          if (pend[t] >= 0 && !issue_pv(t)) { ok = false; break; }
+          const uint32_t qaddr = sbase + C::kQOff + t * C::kQBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / C::kKStep; ++kk) {
+            const uint32_t byte = kk * C::kKStep * C::kEB;  // K offset of this step in bytes
+            const uint32_t chunk = byte / 128, off = byte % 128;
+            const uint64_t adesc = make_sdesc(qaddr + chunk * (128 * 128) + off, 16, 1024);
+            const uint64_t bdesc = make_sdesc(kaddr + chunk * (BN * 128) + off, 16, 1024);
+            if constexpr (FP8) mma_f8_ss(tmem + s_col(t), adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+            else mma_f16_ss(tmem + s_col(t), adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&sh.s_full[t]);
+          ++n[t];
+          pend[t] = k;
+        }
+        if (!ok) break;
+        tc_commit(&sh.k_empty[ks]);
+        // Tiles that skipped this block: flush their pending PV now, so that no V slot is
+        // held past the next block (each V slot is reused two union blocks later).
+        for (int t = 0; t < 2 && ok; ++t)
+          if (!((bits >> t) & 1) && pend[t] >= 0 && !issue_pv(t)) ok = false;
+      }
+      for (int t = 0; t < 2; ++t) {
+        if (ok && pend[t] >= 0 && !issue_pv(t)) ok = false;
+        tc_commit(&sh.o_final[t]);
+      }
+      if (!ok) { record_status(a.status, kStatusTimeout); sh.abort_flag = 1; }
+      // Every MMA of this CTA has completed before TMEM is released (bounded wait).
+      tc_commit(&sh.drain);
+      if (!mbar_wait(&sh.drain, 0)) record_status(a.status, kStatusTimeout);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int t = (warp - 4) / 4;
+    const int r = (warp % 4) * 32 + lane;  // query row of the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
+    const uint32_t s_tm = tmem + lane_base + (t == 0 ? C::kS0 : C::kS1);
+    const uint32_t o_tm = tmem + lane_base + (t == 0 ? C::kO0 : C::kO1);
+    const Tile T = t == 0 ? tl[0] : tl[1];
+    float sl2 = a.scale_log2;
+    if constexpr (FP8) sl2 *= __ldg(a.q_scale + T.h) * __ldg(a.k_scale + g);
+    float m = -INFINITY, l = 0.f;
+    int n = 0;
+    bool ok = true;
+    int i = 0;
+    for (;;) {
+      const int J = next_valid(T.list, T.cnt, i, T.I, a.status, r == 0);
+      if (J < 0) break;
+      const bool got = !sh.abort_flag && mbar_wait(&sh.s_full[t], n & 1);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN; c += 32) tmem_ld32(s_tm + c, s + c);
+      tmem_ld_wait();
+      const bool diag = (J == T.I);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        s[c] = (diag && c > r) ? -INFINITY : s[c] * sl2;
+        mx = fmaxf(mx, s[c]);
+      }
+      // Lazy rescaling: keep the stale max unless the row max grew by more than 2^8, so P
+      // stays <= 256 (exact in fp32 accumulation, in range for bf16 and e4m3).
+      bool rescale = false;
+      float f = 1.f;
+      if (n == 0) {
+        m = mx;
+      } else if (mx > m + 8.f) {
+        f = ex2(m - mx);
+        l *= f;
+        m = mx;
+        rescale = true;
+      }
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      float sum = 0.f;
+      // P = 2^(s - m) in 32-column chunks, packed and written over the S columns of TMEM.
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        if constexpr (FP8) {
+          uint32_t w[8];
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float p0 = ex2(s[c0 + c] - mu), p1 = ex2(s[c0 + c + 1] - mu);
+            const float p2 = ex2(s[c0 + c + 2] - mu), p3 = ex2(s[c0 + c + 3] - mu);
+            sum += (p0 + p1) + (p2 + p3);
+            w[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
+          }
+          tmem_st8(s_tm + c0 / 4, w);
+        } else {
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2(s[c0 + c] - mu), p1 = ex2(s[c0 + c + 1] - mu);
+            sum += p0 + p1;
+            w[c / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(s_tm + c0 / 2, w);
+        }
+      }
+      l += sum;
+      if (rescale) {
+        // PV of the previous block has completed (it precedes S of this block on the tensor
+        // pipe), and the next PV waits for p_full: O can be rescaled in place.
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          tmem_ld32(o_tm + c, o);
+          tmem_ld_wait();
+          uint32_t w[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(o[e] * f);
+          tmem_st32(o_tm + c, w);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sh.p_full[t]);
+      ++n;
+    }
+    // Epilogue: wait for the last PV of this tile, normalise, store.
+    const bool fin = ok && !sh.abort_flag && mbar_wait(&sh.o_final[t], 0);
+    if (__all_sync(0xffffffffu, fin)) {
+      tc_fence_after();
+      if (n > 0) {
+        float inv = (l > 0.f) ? 1.f / l : 0.f;
+        if constexpr (FP8) inv *= __ldg(a.v_scale + g);
+        const bool valid = r < T.nvalid;
+        __nv_bfloat16* orow = a.out + (static_cast<size_t>(T.q_lo + r) * a.Hq + T.h) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          tmem_ld32(o_tm + c, o);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
+              v.y = pack_bf16x2(o[e + 2] * inv, o[e + 3] * inv);
+              v.z = pack_bf16x2(o[e + 4] * inv, o[e + 5] * inv);
+              v.w = pack_bf16x2(o[e + 6] * inv, o[e + 7] * inv);
+              *reinterpret_cast<uint4*>(orow + c + e) = v;
+            }
+          }
+        }
+        if (valid && a.lse != nullptr)
+          a.lse[static_cast<size_t>(T.h) * a.total_tokens + T.q_lo + r] =
+              (l > 0.f) ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      } else if (r < T.nvalid) {
+        // No kept block at all: the row attends to nothing; write zeros / -inf.
+        __nv_bfloat16* orow = a.out + (static_cast<size_t>(T.q_lo + r) * a.Hq + T.h) * D;
+        for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+        if (a.lse != nullptr)
+          a.lse[static_cast<size_t>(T.h) * a.total_tokens + T.q_lo + r] = -INFINITY;
+      }
+    } else {
+      record_status(a.status, kStatusTimeout);
+      sh.abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, heads, d] token-major tensor; box = (one 128-byte chunk of d, 1 head, box_rows rows).
+static bool make_map(CUtensorMap* m, const void* base, bool e4m3, int d, int heads,
+                     long long rows, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  const int eb = e4m3 ? 1 : 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb,
+                           static_cast<cuuint64_t>(d) * heads * eb};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), 1u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int BN, bool FP8, bool PAGED>
+static cudaError_t launch_t(const AttnArgs& a, const AttnLaunch& L, cudaStream_t stream) {
+  using C = AttnCfg<D, BN, FP8>;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, L.q, FP8, D, a.Hq, a.total_tokens, 128) ||
+      !make_map(&mk, L.k, FP8, D, a.Hkv, L.kv_rows, L.seg_rows) ||
+      !make_map(&mv, L.v, FP8, D, a.Hkv, L.kv_rows, L.seg_rows))
+    return cudaErrorInvalidValue;
+  auto kern = attn_kernel<D, BN, FP8, PAGED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  if (a.num_items == 0) return cudaSuccess;
+  kern<<<a.num_items, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn(const AttnArgs& a, const AttnLaunch& L, int block, cudaStream_t stream) {
+  if (L.e4m3) {
+    if (L.d == 128 && block == 128)
+      return L.paged ? launch_t<128, 128, true, true>(a, L, stream)
+                     : launch_t<128, 128, true, false>(a, L, stream);
+    return cudaErrorNotSupported;
+  }
+  if (L.d == 128 && block == 128)
+    return L.paged ? launch_t<128, 128, false, true>(a, L, stream)
+                   : launch_t<128, 128, false, false>(a, L, stream);
+  if (L.d == 64 && block == 64)
+    return L.paged ? launch_t<64, 64, false, true>(a, L, stream)
+                   : launch_t<64, 64, false, false>(a, L, stream);
+  if (L.d == 128 && block == 64)
+    return L.paged ? launch_t<128, 64, false, true>(a, L, stream)
+                   : launch_t<128, 64, false, false>(a, L, stream);
+  if (L.d == 64 && block == 128)
+    return L.paged ? launch_t<64, 128, false, true>(a, L, stream)
+                   : launch_t<64, 128, false, false>(a, L, stream);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace fp

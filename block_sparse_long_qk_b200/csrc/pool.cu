@@ -1,0 +1,127 @@
+// Stage 1: block-mean pooling of Q and K.
+//
+// "FlashPrefill: Instantaneous Pattern Discovery and Thresholding for Ultra-Fast Long-Context
+// Prefilling", technical summary 2.A: keys are averaged per block (block approximation), and
+// the query skeleton is read as block means of Q as well, so that the pooled score of stage 2
+// equals the mean of the raw scaled Q K^T block (the fused 2-D reduction).
+//
+// HBM-bound stream: every CTA owns one (global block, tensor, 2 KB-wide column slice) and
+// its 128 threads each own 16 contiguous bytes of the token row (8 bf16 or 16 e4m3 values),
+// walking the block's tokens with 8 independent 16-byte loads in flight per thread. A warp
+// therefore reads 512 contiguous bytes of one token row per load. Accumulation is fp32.
+#include "fp_common.cuh"
+#include "fp_launch.h"
+
+namespace fp {
+
+constexpr int kPoolThreads = 128;
+
+template <bool E4M3>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
+  constexpr int EPT = E4M3 ? 16 : 8;  // elements per thread (16 bytes)
+  const int gb = blockIdx.x;
+  const bool is_q = static_cast<int>(blockIdx.y) < a.q_slices;
+  const int slice = is_q ? blockIdx.y : blockIdx.y - a.q_slices;
+  const int H = is_q ? a.Hq : a.Hkv;
+  const int cols = H * a.d;
+  const int col = (slice * kPoolThreads + threadIdx.x) * EPT;
+  if (col >= cols) return;
+
+  int b = 0, base = 0, len = a.total_tokens, blk0 = 0;
+  if (a.cu_blocks != nullptr) {
+    b = find_request(a.cu_blocks, a.batch, gb);
+    base = __ldg(a.cu_seqlens + b);
+    len = __ldg(a.cu_seqlens + b + 1) - base;
+    blk0 = __ldg(a.cu_blocks + b);
+  }
+  const int I = gb - blk0;
+  const int t0 = I * a.block;                      // request-local first token
+  const int n = min(a.block, len - t0);            // valid tokens of this block
+  const uint8_t* src = is_q ? a.q : a.k;
+  const bool paged = (!is_q) && a.page_table != nullptr;
+  const size_t row_bytes = static_cast<size_t>(cols) * (E4M3 ? 1 : 2);
+  const size_t col_bytes = static_cast<size_t>(col) * (E4M3 ? 1 : 2);
+
+  float acc[EPT];
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) acc[i] = 0.f;
+
+  // Token row r of the block; nullptr for a paged token whose page entry is out of range.
+  auto row_ptr = [&](int r) -> const int4* {
+    size_t row;
+    if (paged) {
+      const int tl = t0 + r;
+      const int lp = tl / a.page_size;
+      if (lp >= a.max_pages) return nullptr;
+      const int page = __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp);
+      if (page < 0 || page >= a.num_pages) return nullptr;
+      row = static_cast<size_t>(page) * a.page_size + (tl % a.page_size);
+    } else {
+      row = static_cast<size_t>(base) + t0 + r;
+    }
+    return reinterpret_cast<const int4*>(src + row * row_bytes + col_bytes);
+  };
+  auto load = [&](int r) -> int4 {
+    const int4* p = row_ptr(r);
+    return p ? __ldcs(p) : make_int4(0, 0, 0, 0);
+  };
+
+  auto accumulate = [&](int4 v) {
+    if constexpr (E4M3) {
+      const __nv_fp8x2_storage_t* p2 = reinterpret_cast<const __nv_fp8x2_storage_t*>(&v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(p2[i], __NV_E4M3);
+        float2 f = __half22float2(*reinterpret_cast<__half2*>(&h));
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    } else {
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(p2[i]);
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
+    }
+  };
+
+  int r = 0;
+  for (; r + 8 <= n; r += 8) {
+    int4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = load(r + u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) accumulate(v[u]);
+  }
+  for (; r < n; ++r) accumulate(load(r));
+
+  const int h = col / a.d;
+  const int c = col % a.d;
+  float s = 1.f / static_cast<float>(n);
+  const float* scale = is_q ? a.q_scale : a.k_scale;
+  if (scale != nullptr) s *= __ldg(scale + h);
+  float* dst = (is_q ? a.q_pool : a.k_pool) +
+               (static_cast<size_t>(h) * a.total_blocks + gb) * a.d + c;
+#pragma unroll
+  for (int i = 0; i < EPT; i += 4)
+    *reinterpret_cast<float4*>(dst + i) =
+        make_float4(acc[i] * s, acc[i + 1] * s, acc[i + 2] * s, acc[i + 3] * s);
+}
+
+cudaError_t launch_pool(const PoolArgs& in, bool e4m3, cudaStream_t stream) {
+  PoolArgs a = in;
+  const int ept = e4m3 ? 16 : 8;
+  const int per_cta = kPoolThreads * ept;
+  a.q_slices = (a.Hq * a.d + per_cta - 1) / per_cta;
+  const int k_slices = (a.Hkv * a.d + per_cta - 1) / per_cta;
+  dim3 grid(a.total_blocks, a.q_slices + k_slices);
+  if (e4m3)
+    pool_kernel<true><<<grid, kPoolThreads, 0, stream>>>(a);
+  else
+    pool_kernel<false><<<grid, kPoolThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fp

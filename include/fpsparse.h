@@ -1,0 +1,177 @@
+/*
+ * fpsparse -- block-sparse causal prefill attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libfpsparse.so. The three stages of the method, each one CUDA kernel:
+ *
+ *   fp_pool_qk               block means of Q and K            ("FlashPrefill: Instantaneous
+ *                            Pattern Discovery and Thresholding for Ultra-Fast Long-Context
+ *                            Prefilling", technical summary 2.A, block approximation and the
+ *                            fused 2-D reduction)
+ *   fp_build_block_mask      pooled block scores, max-based dynamic threshold, KV-block mask
+ *                            and index lists                    (same page, 2.B)
+ *   fp_sparse_prefill_attn   causal attention over the kept KV blocks only, index-based
+ *                            physical skip                      (same page, 2.C; GQA packing,
+ *                            FP8 and paged KV with continuous batching from "FlashPrefill V2:
+ *                            Block-Sparse Prefill Attention for Long-Context LLM Serving",
+ *                            Abstract)
+ *   fp_sparse_prefill_attn_paged   the same with K/V read through a page table
+ *
+ * Conventions for every call:
+ *  - Every pointer argument is a DEVICE pointer unless its comment says "host". The caller
+ *    owns all memory; the library allocates nothing on these paths. Inputs are read only.
+ *  - Token-major activations: Q is [T, Hq, d], K and V are [T, Hkv, d], row-major and
+ *    contiguous (element (t, h, c) at ((t * H) + h) * d + c). T is the total token count of
+ *    the batch. Query head h reads KV head h / (Hq / Hkv) (grouped-query attention).
+ *  - Varlen batches: cu_seqlens is int32 [batch + 1] (cu[0] = 0, cu[batch] = T, ascending)
+ *    and cu_blocks is int32 [batch + 1] with cu_blocks[b+1] - cu_blocks[b] =
+ *    ceil((cu[b+1] - cu[b]) / block). Blocks restart at each request's first token; a
+ *    request's last block may be partial. For one sequence pass batch = 1 and both pointers
+ *    NULL. "Global block" Ig indexes the blocks of all requests in order (0 .. total_blocks).
+ *  - dtype is FP_DTYPE_BF16 or FP_DTYPE_E4M3. For e4m3 storage the real value of an element
+ *    is code * scale[head], with one float32 scale per head (q_scale [Hq], k_scale and
+ *    v_scale [Hkv]); for bf16 the scale pointers must be NULL.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ *    and is asynchronous. Argument errors are reported before anything is enqueued.
+ *  - Return value: FP_OK (0) or a negative FP_ERR_* code; fp_last_error_string() then holds
+ *    a message for the calling thread. Nothing throws across this boundary.
+ */
+#ifndef FPSPARSE_H_
+#define FPSPARSE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP_OK 0
+#define FP_ERR_INVALID_ARG (-1)  /* a size, pointer or alignment the call cannot accept */
+#define FP_ERR_UNSUPPORTED (-2)  /* a valid configuration that this build does not cover */
+#define FP_ERR_CUDA (-3)         /* a CUDA runtime or driver call failed */
+#define FP_ERR_TIMEOUT (-4)      /* a kernel pipeline wait ran out (reported by fp_check_status) */
+#define FP_ERR_BAD_INDEX (-5)    /* an index list or page table entry out of range (fp_check_status) */
+
+#define FP_DTYPE_BF16 0
+#define FP_DTYPE_E4M3 1
+
+#define FP_FORCE_FIRST 1 /* always keep KV block 0 of every row */
+#define FP_FORCE_DIAG 2  /* always keep the diagonal KV block J = I */
+
+/* Library version, e.g. 100 for 0.1.0. */
+int fp_version(void);
+
+/* Message describing the last error returned on the calling thread ("" if none). */
+const char* fp_last_error_string(void);
+
+/*
+ * Stage 1: block-mean pooling ("FlashPrefill: Instantaneous Pattern Discovery ...",
+ * technical summary 2.A: keys averaged per block; queries read the same way).
+ *
+ *   q_pool[h, Ig, :] = mean over the valid tokens i of block Ig of Q[i, h, :] * q_scale[h]
+ *   k_pool[g, Ig, :] = mean over the valid tokens j of block Ig of K[j, g, :] * k_scale[g]
+ *
+ * q, k       Q [T, Hq, d], K [T, Hkv, d] in `dtype`; with k_page_table != NULL, k is instead
+ *            a paged cache [num_pages, page_size, Hkv, d] and token t of request b lives in
+ *            page k_page_table[b * max_pages + t / page_size], slot t % page_size; entries
+ *            outside [0, num_pages) and pages past max_pages are not read (those tokens count
+ *            as zeros).
+ * q_pool     float32 [Hq, total_blocks, d] (written)
+ * k_pool     float32 [Hkv, total_blocks, d] (written)
+ * Supported: d in {64, 128}; block in {64, 128}; Hq % Hkv == 0; page_size a multiple of 16
+ * that divides block. Q and K must be 16-byte aligned.
+ */
+int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
+               const float* k_scale, const int32_t* cu_seqlens, const int32_t* cu_blocks,
+               int batch, int total_tokens, int total_blocks, int Hq, int Hkv, int d,
+               int block, const int32_t* k_page_table, int page_size, int max_pages,
+               int num_pages, float* q_pool, float* k_pool, void* stream);
+
+/*
+ * Stage 2: pooled block scores and the max-based dynamic threshold ("FlashPrefill:
+ * Instantaneous Pattern Discovery ...", technical summary 2.B: thresh_I = alpha *
+ * max_{J<=I} Score_{I,J}, no sort and no top-k).
+ *
+ * Per head h and request-local query block I (global row Ig), over the causal blocks J <= I
+ * of the same request:
+ *   s_J  = scale * dot(q_pool[h, Ig], k_pool[h / (Hq/Hkv), cu_blocks[b] + J])   (float32)
+ *   keep J  iff  s_J - max_J s_J >= ln(alpha)          (= softmax(s)_J >= alpha * max softmax)
+ *           or (flags & FP_FORCE_FIRST and J == 0) or (flags & FP_FORCE_DIAG and J == I).
+ * alpha in [0, 1]; alpha = 0 keeps every causal block.
+ *
+ * mask_bits  uint32 [Hq, total_blocks, words], words = ceil(max_blocks / 32): bit J % 32 of
+ *            word J / 32 is set iff block J is kept (bits above I are 0). May be NULL.
+ * kv_cnt     int32 [Hq, total_blocks]: number of kept blocks of the row
+ * kv_idx     int32 [Hq, total_blocks, max_blocks]: the kept request-local block indices in
+ *            ascending order in the first kv_cnt entries (the rest is left untouched)
+ * max_blocks largest per-request block count (host int)
+ */
+int fp_build_block_mask(const float* q_pool, const float* k_pool, const int32_t* cu_blocks,
+                        int batch, int total_blocks, int max_blocks, int Hq, int Hkv, int d,
+                        float alpha, float scale, int flags, uint32_t* mask_bits,
+                        int32_t* kv_cnt, int32_t* kv_idx, void* stream);
+
+/*
+ * Stage 3: causal attention over the kept KV blocks only ("FlashPrefill: Instantaneous
+ * Pattern Discovery ...", technical summary 2.C, index-based physical skip; GQA packing and
+ * FP8 as in "FlashPrefill V2 ...", Abstract).
+ *
+ *   out[i, h, :] = sum_j softmax_j(scale * q_i . k_j) v_j   over the keys j <= i of the same
+ *                  request whose block J = (j - cu[b]) / block is listed in
+ *                  kv_idx[h, Ig, 0 .. kv_cnt[h, Ig]), Ig the global block of query i.
+ *   lse[h, i]    = ln sum_j exp(scale * q_i . k_j) over the same keys (may be NULL).
+ *
+ * Index lists must be ascending, request-local and causal (0 <= J <= I); entries outside that
+ * range are skipped and reported as FP_ERR_BAD_INDEX by fp_check_status.
+ * q, k, v    as in fp_pool_qk (e4m3: per-head scales; the output is always bf16)
+ * out        bf16 [T, Hq, d] (written)
+ * lse        float32 [Hq, T] or NULL
+ * workspace  at least fp_workspace_size() bytes of device memory, 256-byte aligned, holding
+ *            the status word that fp_check_status reads. Concurrent calls need distinct
+ *            workspaces.
+ * Supported: d in {64, 128}; block in {64, 128} (e4m3: d = 128, block = 128);
+ * Hq % Hkv == 0. Q, K, V must be 16-byte aligned.
+ */
+int fp_sparse_prefill_attn(const void* q, const void* k, const void* v, int dtype,
+                           const float* q_scale, const float* k_scale, const float* v_scale,
+                           const int32_t* cu_seqlens, const int32_t* cu_blocks, int batch,
+                           int total_tokens, int total_blocks, int max_blocks, int Hq,
+                           int Hkv, int d, int block, float scale, const int32_t* kv_cnt,
+                           const int32_t* kv_idx, void* out, float* lse, void* workspace,
+                           void* stream);
+
+/*
+ * Stage 3 with a paged KV cache and a continuous (varlen) batch ("FlashPrefill V2 ...",
+ * Abstract: paged KV cache and continuous batching). Same definition as
+ * fp_sparse_prefill_attn; K and V are read as caches [num_pages, page_size, Hkv, d] through
+ * page_table int32 [batch, max_pages] (entry -1 or >= num_pages is FP_ERR_BAD_INDEX when it
+ * would be read). page_size must be a multiple of 16 that divides block. Queries are
+ * contiguous [T, Hq, d] with cu_seqlens (query length = KV length: prefill from scratch).
+ */
+int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void* v_cache,
+                                 int dtype, const float* q_scale, const float* k_scale,
+                                 const float* v_scale, const int32_t* cu_seqlens,
+                                 const int32_t* cu_blocks, int batch, int total_tokens,
+                                 int total_blocks, int max_blocks, int Hq, int Hkv, int d,
+                                 int block, const int32_t* page_table, int page_size,
+                                 int max_pages, int num_pages, float scale,
+                                 const int32_t* kv_cnt, const int32_t* kv_idx, void* out,
+                                 float* lse, void* workspace, void* stream);
+
+/* Bytes of device workspace the attention calls need (a fixed small size). */
+size_t fp_workspace_size(void);
+
+/*
+ * Waits for `stream`, reads and clears the status word in `workspace`, and returns FP_OK,
+ * FP_ERR_TIMEOUT or FP_ERR_BAD_INDEX (or FP_ERR_CUDA if the stream itself failed).
+ * The workspace must have been zeroed once before its first use (e.g. cudaMemset).
+ * A recorded timeout is sticky: attention launches on that workspace do no work (their CTAs
+ * exit at once) until this call has cleared it.
+ */
+int fp_check_status(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FPSPARSE_H_ */

@@ -1,0 +1,59 @@
+"""The C-ABI library loads, exports every symbol its header declares, and rejects bad
+arguments on the host before touching a GPU (no compute call here)."""
+import ctypes
+
+import pytest
+
+import block_sparse_long_qk_b200 as fp
+
+
+def test_library_exports_every_header_symbol():
+    lib = fp.library()
+    names = fp.header_symbols()
+    assert "fp_pool_qk" in names and "fp_sparse_prefill_attn_paged" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(fp._SIGNATURES), "binding lacks a signature for a header symbol"
+
+
+def test_version_and_workspace():
+    lib = fp.library()
+    assert lib.fp_version() >= 100
+    assert lib.fp_workspace_size() >= 4
+
+
+def _bad_attn(**over):
+    """Arguments of a well-formed single-sequence attention call with fake pointers; only
+    host-side validation runs for the failing cases below."""
+    a = dict(q=16, k=16, v=16, dtype=0, qs=None, ks=None, vs=None, cu=None, cb=None, batch=1,
+             T=256, tb=2, mb=2, Hq=8, Hkv=2, d=128, block=128, scale=0.1, cnt=16, idx=16,
+             out=16, lse=None, ws=256, stream=None)
+    a.update(over)
+    lib = fp.library()
+    return lib.fp_sparse_prefill_attn(*[a[k] for k in (
+        "q", "k", "v", "dtype", "qs", "ks", "vs", "cu", "cb", "batch", "T", "tb", "mb", "Hq",
+        "Hkv", "d", "block", "scale", "cnt", "idx", "out", "lse", "ws", "stream")])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(dtype=7), -1),             # unknown dtype
+    (dict(Hq=6, Hkv=4), -1),         # Hq not a multiple of Hkv
+    (dict(d=96), -2),                # unsupported head dim
+    (dict(block=32), -2),            # unsupported block
+    (dict(tb=3), -1),                # total_blocks != ceil(T / block)
+    (dict(q=8), -1),                 # misaligned pointer
+    (dict(ws=128), -1),              # misaligned workspace
+    (dict(dtype=1), -1),             # e4m3 without scales
+    (dict(batch=2), -1),             # varlen without cu arrays
+])
+def test_attention_rejects_bad_arguments(over, code):
+    assert _bad_attn(**over) == code
+    assert fp.library().fp_last_error_string()
+
+
+def test_mask_rejects_alpha_out_of_range():
+    lib = fp.library()
+    rc = lib.fp_build_block_mask(16, 16, None, 1, 4, 4, 8, 2, 128, 1.5, 0.1, 3, None, 16, 16,
+                                 None)
+    assert rc == -1
+    assert b"alpha" in lib.fp_last_error_string()

@@ -1,0 +1,185 @@
+"""GPU parity of the three kernels against the fp64 oracle (through the C ABI).
+
+Every case draws seeded synthetic inputs, runs the CUDA path, and compares element by
+element with the oracle on the same inputs: pooled means, the block mask (bit-identical
+up to near-threshold blocks), and the attention output computed from the oracle's own keep
+set (index lists written on the host from that set), so that no oracle input ever comes
+from the CUDA path.
+"""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_qk_b200 as fp
+from block_sparse_long_qk_b200 import synthetic as S
+
+from _parity import (TOL, OracleRun, attn_errors, bits_to_keeps, device_inputs, keep_to_lists,
+                     lists_to_keeps, mask_mismatches)
+
+pytestmark = pytest.mark.gpu
+
+W = S.WORKLOADS
+
+
+def _case(name):
+    """Small workloads: several tiles, ragged tails, every kernel variant."""
+    base = W["llama32k"]
+    cases = {
+        "tiny": (W["tiny"], None, 0.1),
+        "tiny_a09": (W["tiny"], None, 0.9),
+        "gqa_ragged": (dataclasses.replace(base, Hq=8, Hkv=2, structure="band"), (1000,), 0.1),
+        "gqa_ragged_a05": (dataclasses.replace(base, Hq=8, Hkv=2, structure="iid"), (1000,), 0.5),
+        "varlen": (dataclasses.replace(base, Hq=8, Hkv=2, structure="iid"), (300, 129, 640), 0.5),
+        "paged": (dataclasses.replace(W["paged"], Hq=8, Hkv=2, structure="iid"),
+                  (300, 129, 640), 0.5),
+        "fp8": (dataclasses.replace(W["fp8_128k"], Hq=8, Hkv=2, structure="iid"), (1000,), 0.5),
+        "mha_d128": (dataclasses.replace(base, Hq=4, Hkv=4, structure="iid"), (700,), 0.5),
+        "dense_alpha0": (dataclasses.replace(base, Hq=4, Hkv=2, structure="iid"), (600,), 0.0),
+        "d128_b64": (dataclasses.replace(base, Hq=4, Hkv=2, block=64, structure="iid"),
+                     (500,), 0.5),
+        "d64_b128": (dataclasses.replace(base, Hq=4, Hkv=2, d=64, structure="iid"), (500,), 0.5),
+    }
+    w, seqlens, alpha = cases[name]
+    return S.make_inputs(w, seed=7, seqlens=seqlens), alpha
+
+
+SMALL = ["tiny", "tiny_a09", "gqa_ragged", "gqa_ragged_a05", "varlen", "paged", "fp8",
+         "mha_d128", "dense_alpha0", "d128_b64", "d64_b128"]
+
+
+def _batch(inp, dev):
+    return fp.Batch.make(inp.workload.seqlens, inp.workload.block, dev)
+
+
+def _paged(inp, dev):
+    if not inp.workload.page_size:
+        return None
+    return fp.PagedKV(inp.k_cache.to(dev), inp.v_cache.to(dev), inp.page_table.to(dev))
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_pool_and_mask_match_oracle(name, cuda_device):
+    inp, alpha = _case(name)
+    run = OracleRun(inp, alpha)
+    q, k, v, sc = device_inputs(inp, cuda_device)
+    b = _batch(inp, cuda_device)
+    qp, kp = fp.pool_qk(q, k, inp.workload.block, batch=b, q_scale=sc["q_scale"],
+                        k_scale=sc["k_scale"], paged=_paged(inp, cuda_device))
+    torch.cuda.synchronize()
+    for got, ref in ((qp, run.q_pool), (kp, run.k_pool)):
+        g = got.cpu().double().numpy()
+        assert np.abs(g - ref).max() <= 1e-5 * max(1.0, np.abs(ref).max())
+    bits, cnt, idx = fp.build_block_mask(qp, kp, alpha, block=inp.workload.block, batch=b)
+    torch.cuda.synchronize()
+    gk = bits_to_keeps(bits, run)
+    bad, ex, tot = mask_mismatches(gk, run)
+    assert bad == 0, f"{bad} non-exempt mask mismatches of {tot}"
+    assert ex <= max(2, tot // 1000)
+    # the index lists say the same as the bits
+    lk = lists_to_keeps(cnt, idx, run)
+    for a_, b_ in zip(gk, lk):
+        assert np.array_equal(a_, b_)
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_attention_matches_oracle(name, cuda_device):
+    inp, alpha = _case(name)
+    w = inp.workload
+    run = OracleRun(inp, alpha)
+    ref, ref_lse = run.attention()
+    cnt, idx = keep_to_lists(run.keeps, w.Hq)
+    q, k, v, sc = device_inputs(inp, cuda_device)
+    b = _batch(inp, cuda_device)
+    kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"],
+              return_lse=True)
+    if w.page_size:
+        out, lse = fp.sparse_prefill_attn_paged(q, _paged(inp, cuda_device), cnt.to(cuda_device),
+                                                idx.to(cuda_device), b, **kw)
+    else:
+        out, lse = fp.sparse_prefill_attn(q, k, v, cnt.to(cuda_device), idx.to(cuda_device),
+                                          w.block, batch=b, **kw)
+    fp.check_status(cuda_device)
+    amax, rel = attn_errors(out, ref)
+    tol = TOL[w.dtype]
+    assert amax <= tol[0] and rel <= tol[1], (amax, rel)
+    dl = np.abs(lse.cpu().double().numpy() - ref_lse)
+    assert np.nanmax(dl) <= (2e-3 if w.dtype == "bf16" else 3e-2)
+
+
+def test_skipped_blocks_are_never_read(cuda_device):
+    """Physical skip: query blocks 3..7 do not keep KV blocks 1 and 2, whose K/V rows are then
+    poisoned with NaN. Those query blocks' outputs stay finite and bit-identical."""
+    w = dataclasses.replace(W["llama32k"], Hq=4, Hkv=2, structure="iid")
+    inp = S.make_inputs(w, seed=3, seqlens=(1024,))
+    keep = np.tril(np.ones((4, 8, 8), dtype=bool))
+    keep[:, 3:, 1:3] = False
+    cnt, idx = keep_to_lists([keep], 4)
+    cnt, idx = cnt.to(cuda_device), idx.to(cuda_device)
+    q, k, v, _ = device_inputs(inp, cuda_device)
+    out0, _ = fp.sparse_prefill_attn(q, k, v, cnt, idx, 128)
+    kp, vp = k.clone(), v.clone()
+    kp[128:384] = float("nan")
+    vp[128:384] = float("nan")
+    out1, _ = fp.sparse_prefill_attn(q, kp, vp, cnt, idx, 128)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out1[384:].float()).all()
+    assert torch.equal(out0[384:], out1[384:])
+
+
+def test_bad_index_is_reported_not_read(cuda_device):
+    w = dataclasses.replace(W["llama32k"], Hq=2, Hkv=1, structure="iid")
+    inp = S.make_inputs(w, seed=4, seqlens=(512,))
+    keep = np.tril(np.ones((2, 4, 4), dtype=bool))
+    cnt, idx = keep_to_lists([keep], 2)
+    idx[0, 1, 1] = 3   # a non-causal block for query block 1
+    q, k, v, _ = device_inputs(inp, cuda_device)
+    fp.sparse_prefill_attn(q, k, v, cnt.to(cuda_device), idx.to(cuda_device), 128)
+    with pytest.raises(fp.FpError) as e:
+        fp.check_status(cuda_device)
+    assert e.value.code == -5
+    fp.check_status(cuda_device)   # cleared
+
+
+def _full_size(name, cuda_device, n_rows=48):
+    inp = S.make_inputs(name)
+    w = inp.workload
+    run = OracleRun(inp, w.alpha)
+    q, k, v, sc = device_inputs(inp, cuda_device)
+    b = _batch(inp, cuda_device)
+    paged = _paged(inp, cuda_device)
+    qp, kp = fp.pool_qk(q, k, w.block, batch=b, q_scale=sc["q_scale"], k_scale=sc["k_scale"],
+                        paged=paged)
+    bits, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b)
+    kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"])
+    if paged is not None:
+        out, _ = fp.sparse_prefill_attn_paged(q, paged, cnt, idx, b, **kw)
+    else:
+        out, _ = fp.sparse_prefill_attn(q, k, v, cnt, idx, w.block, batch=b, **kw)
+    fp.check_status(cuda_device)
+    gk = bits_to_keeps(bits, run)
+    bad, ex, tot = mask_mismatches(gk, run)
+    assert bad == 0 and ex <= max(4, tot // 100000), (bad, ex, tot)
+    # sampled (head, query block) rows whose GPU and oracle masks agree
+    rng = np.random.default_rng(11)
+    rows = []
+    while len(rows) < n_rows:
+        h = int(rng.integers(w.Hq))
+        Ig = int(rng.integers(run.off[-1]))
+        r = int(np.searchsorted(run.off, Ig, side="right") - 1)
+        I = Ig - run.off[r]
+        if np.array_equal(gk[r][h, I], run.keeps[r][h, I]):
+            rows.append((h, Ig))
+    rows.append((0, run.off[-1] - 1))
+    ref, _ = run.attention(rows=rows)
+    amax, rel = attn_errors(out, ref)
+    tol = TOL[w.dtype]
+    assert amax <= tol[0] and rel <= tol[1], (amax, rel)
+    return run
+
+
+@pytest.mark.parametrize("name", ["llama32k", "llama128k", "fp8_128k", "paged"])
+def test_full_size_workloads(name, cuda_device):
+    _full_size(name, cuda_device)
