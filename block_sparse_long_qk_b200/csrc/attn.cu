@@ -335,12 +335,14 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < BN; c += 32) tmem_ld32(s_tm + c, s + c);
       tmem_ld_wait();
       const bool diag = (J == T.I);
-      float mx = -INFINITY;
+      if (diag) {  // causal mask inside the diagonal block: key c > query r
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        s[c] = (diag && c > r) ? -INFINITY : s[c] * sl2;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < BN; ++c) s[c] = (c > r) ? -INFINITY : s[c];
       }
+      float mraw = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) mraw = fmax3(mraw, s[c], s[c + 1]);
+      const float mx = mraw * sl2;  // sl2 > 0: the max commutes with the scaling
       // Lazy rescaling: keep the stale max unless the row max grew by more than 2^8, so P
       // stays <= 256 (exact in fp32 accumulation, in range for bf16 and e4m3).
       bool rescale = false;
@@ -354,33 +356,47 @@ __global__ void __launch_bounds__(384, 1)
         rescale = true;
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
-      float sum = 0.f;
-      // P = 2^(s - m) in 32-column chunks, packed and written over the S columns of TMEM.
+      const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-mu, -mu);
+      float2 sum2 = make_float2(0.f, 0.f);
+      // P = 2^(s * sl2 - m) in 32-column chunks, packed and written over the S columns of TMEM.
+      // Off the diagonal, one column pair in four takes the FMA-pipe polynomial instead of
+      // MUFU ex2, so the exponentials do not outrun the tensor core on the MUFU unit.
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += 32) {
+        float2 pp[16];
+        if (diag) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 x = ffma2(make_float2(s[c0 + c], s[c0 + c + 1]), sc2, nm2);
+            pp[c / 2] = make_float2(ex2(x.x), ex2(x.y));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 x = ffma2(make_float2(s[c0 + c], s[c0 + c + 1]), sc2, nm2);
+            pp[c / 2] = ((c / 2) % 4 == 3) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) sum2 = fadd2(sum2, pp[e]);
         if constexpr (FP8) {
           uint32_t w[8];
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            const float p0 = ex2(s[c0 + c] - mu), p1 = ex2(s[c0 + c + 1] - mu);
-            const float p2 = ex2(s[c0 + c + 2] - mu), p3 = ex2(s[c0 + c + 3] - mu);
-            sum += (p0 + p1) + (p2 + p3);
-            w[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
-          }
+          for (int e = 0; e < 8; ++e)
+            w[e] = pack_e4m3x4(pp[2 * e].x, pp[2 * e].y, pp[2 * e + 1].x, pp[2 * e + 1].y);
           tmem_st8(s_tm + c0 / 4, w);
         } else {
           uint32_t w[16];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float p0 = ex2(s[c0 + c] - mu), p1 = ex2(s[c0 + c + 1] - mu);
-            sum += p0 + p1;
-            w[c / 2] = pack_bf16x2(p0, p1);
-          }
+          for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(pp[e].x, pp[e].y);
           tmem_st16(s_tm + c0 / 2, w);
         }
       }
+      const float sum = sum2.x + sum2.y;
       l += sum;
-      if (rescale) {
+      // tcgen05.ld/st are warp-collective: when any row of the warp rescales, the whole warp
+      // runs the pass (f = 1 for rows that keep their max).
+      if (__any_sync(0xffffffffu, rescale)) {
         // PV of the previous block has completed (it precedes S of this block on the tensor
         // pipe), and the next PV waits for p_full: O can be rescaled in place.
 #pragma unroll 1

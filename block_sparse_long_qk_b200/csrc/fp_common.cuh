@@ -74,7 +74,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    // The iteration cap bounds the wait even if the global timer were not advancing.
+    if ((i & 63u) == 0u && (globaltimer_ns() - t0 > kWaitLimitNs || i > (1u << 26))) return false;
   }
 }
 
@@ -263,6 +264,53 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2 instructions) -------------------------------------------
+__device__ __forceinline__ uint64_t f2_bits(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
+__device__ __forceinline__ float2 bits_f2(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 fadd2_rm(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe (offloads the MUFU unit). Range reduction x = n + f with
+// n = floor(x) taken by adding 1.5 * 2^23 under round-toward-minus-infinity, a cubic for 2^f on
+// [0, 1) (coefficients from exp2_poly_fit.py: Remez fit of the relative error with p(0) = 1,
+// p(1) = 2; max relative error 1.03e-4), and 2^n applied by adding n to the exponent field.
+// Inputs are clamped to >= -126 (results below 2^-126 come out as 2^-126 instead of 0); not for
+// -inf inputs that must give 0.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = fadd2_rm(x, make_float2(kMagic, kMagic));
+  const float2 nf = fadd2(t, make_float2(-kMagic, -kMagic));
+  const float2 f = ffma2(nf, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(0.07826796919107437f, 0.07826796919107437f), f,
+                   make_float2(0.226307675242424f, 0.226307675242424f));
+  p = ffma2(p, f, make_float2(0.6954243183135986f, 0.6954243183135986f));
+  p = ffma2(p, f, make_float2(1.f, 1.f));
+  const uint32_t lo = __float_as_uint(p.x) + __float_as_uint(t.x) * 8388608u;  // + n << 23
+  const uint32_t hi = __float_as_uint(p.y) + __float_as_uint(t.y) * 8388608u;
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
 }
 
 // Four floats -> four e4m3 codes (round to nearest even, saturating), first in the low byte.

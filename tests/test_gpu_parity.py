@@ -129,6 +129,63 @@ def test_skipped_blocks_are_never_read(cuda_device):
     assert torch.equal(out0[384:], out1[384:])
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_lane_divergent_rescale(dtype, cuda_device):
+    """Even query rows of the last block see a score jump of ~10 log2 units at KV block 2 (the
+    running max is rescaled), odd rows do not: rows of one warp take different paths through
+    the lazy O rescale and must still match the oracle."""
+    L, d = 512, 128
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn(L, 2, d, generator=g) * 0.1
+    k = torch.randn(L, 1, d, generator=g) * 0.1
+    v = torch.randn(L, 1, d, generator=g)
+    u = torch.zeros(d)
+    u[3] = 1.0
+    k[256:384, 0] += 9.0 * u
+    q[384::2, :] += 9.0 * u
+    w = dataclasses.replace(W["llama32k"], Hq=2, Hkv=1, seqlens=(L,), dtype=dtype)
+    inp = S.Inputs(w, q, k, v, torch.tensor([0, L], dtype=torch.int32))
+    if dtype == "e4m3":
+        inp.q, inp.q_scale = S.quantize_e4m3(q)
+        inp.k, inp.k_scale = S.quantize_e4m3(k)
+        inp.v, inp.v_scale = S.quantize_e4m3(v)
+    else:
+        inp.q, inp.k, inp.v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    run = OracleRun(inp, 0.0)        # every causal block kept, ascending order 0, 1, 2, 3
+    ref, _ = run.attention()
+    cnt, idx = keep_to_lists(run.keeps, 2)
+    dq, dk, dv, sc = device_inputs(inp, cuda_device)
+    out, _ = fp.sparse_prefill_attn(dq, dk, dv, cnt.to(cuda_device), idx.to(cuda_device), 128,
+                                    q_scale=sc["q_scale"], k_scale=sc["k_scale"],
+                                    v_scale=sc["v_scale"])
+    fp.check_status(cuda_device)
+    amax, rel = attn_errors(out, ref)
+    tol = TOL[dtype]
+    assert amax <= tol[0] and rel <= tol[1], (amax, rel)
+
+
+def test_band_workload_16k(cuda_device):
+    """The 128K recipe (vertical stripes + local band, alpha 0.1) at 16K tokens: realistic
+    sparse lists whose two heads per CTA differ, many CTA waves, full pipeline."""
+    w = dataclasses.replace(W["llama128k"], seqlens=(16384,))
+    inp = S.make_inputs(w, seed=31)
+    run = OracleRun(inp, w.alpha)
+    q, k, v, _ = device_inputs(inp, cuda_device)
+    b = _batch(inp, cuda_device)
+    qp, kp = fp.pool_qk(q, k, w.block, batch=b)
+    bits, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b)
+    out, _ = fp.sparse_prefill_attn(q, k, v, cnt, idx, w.block, batch=b)
+    fp.check_status(cuda_device)
+    gk = bits_to_keeps(bits, run)
+    bad, ex, tot = mask_mismatches(gk, run)
+    assert bad == 0 and ex <= max(4, tot // 10000), (bad, ex, tot)
+    rows = [(h, I) for h in range(w.Hq) for I in range(0, 128, 9)
+            if np.array_equal(gk[0][h, I], run.keeps[0][h, I])]
+    ref, _ = run.attention(rows=rows)
+    amax, rel = attn_errors(out, ref)
+    assert amax <= TOL["bf16"][0] and rel <= TOL["bf16"][1], (amax, rel)
+
+
 def test_bad_index_is_reported_not_read(cuda_device):
     w = dataclasses.replace(W["llama32k"], Hq=2, Hkv=1, structure="iid")
     inp = S.make_inputs(w, seed=4, seqlens=(512,))
