@@ -28,7 +28,8 @@ import torch
 
 __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_attn",
            "sparse_prefill_attn_paged", "sparse_prefill", "check_status", "workspace",
-           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "header_symbols"]
+           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "header_symbols",
+           "pool_and_mask_noalloc"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfpsparse.so")
@@ -55,6 +56,8 @@ _SIGNATURES = {
                                           _i, _i, _i, _i, _p, _i, _i, _i, _f, _p, _p, _p, _p,
                                           _p, _p]),
     "fp_check_status": (_i, [_p, _p]),
+    "fp_pool_and_mask_noalloc": (_i, [_p, _p, _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
+                                      _i, _p, _i, _i, _i, _f, _f, _i, _p, _p, _p, _p]),
 }
 
 
@@ -301,3 +304,34 @@ def sparse_prefill(q, k=None, v=None, alpha=0.1, block=128, *, batch: Batch | No
                                        q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,
                                        return_lse=return_lse)
     return out, lse, kv_cnt, kv_idx
+
+
+def pool_and_mask_noalloc(q, k, alpha=0.1, block=128, *, batch: Batch | None = None,
+                          scale=None, q_scale=None, k_scale=None, paged: PagedKV | None = None,
+                          flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True):
+    """``pool_qk`` + ``build_block_mask`` with the pooled means kept in the library's static
+    device scratch (for callers that cannot allocate them). Returns (mask_bits or None,
+    kv_cnt, kv_idx); the output tensors are allocated here by torch for convenience."""
+    T, Hq, d = q.shape
+    kk = paged.k_cache if paged is not None else k
+    Hkv = kk.shape[-2]
+    b = _batch_for(q, block, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dev = q.device
+    words = (b.max_blocks + 31) // 32
+    bits = torch.zeros((Hq, b.total_blocks, words), dtype=torch.int32, device=dev) \
+        if mask_bits else None
+    kv_cnt = torch.empty((Hq, b.total_blocks), dtype=torch.int32, device=dev)
+    kv_idx = torch.empty((Hq, b.total_blocks, b.max_blocks), dtype=torch.int32, device=dev)
+    cu, cb = b._ptrs()
+    if paged is not None and cu is None:
+        cu, cb = _ptr(b.cu_seqlens), _ptr(b.cu_blocks)
+    pt = paged.page_table if paged is not None else None
+    _check(library().fp_pool_and_mask_noalloc(
+        _ptr(q), _ptr(kk), _dtype_code(q), _ptr(q_scale), _ptr(k_scale), cu, cb, b.size, T,
+        b.total_blocks, b.max_blocks, Hq, Hkv, d, block, _ptr(pt),
+        paged.page_size if paged else 0, pt.shape[1] if pt is not None else 0,
+        kk.shape[0] if pt is not None else 0, float(alpha), float(scale), int(flags),
+        _ptr(bits), _ptr(kv_cnt), _ptr(kv_idx), _stream(dev)))
+    return bits, kv_cnt, kv_idx

@@ -59,6 +59,18 @@ int check_common(int dtype, const float* qs, const float* ks, const float* vs, b
 
 }  // namespace
 
+namespace fp {
+int set_error(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+}  // namespace fp
+
 extern "C" {
 
 int fp_version(void) { return 100; }

@@ -66,4 +66,7 @@ cudaError_t launch_mask(const MaskArgs& a, cudaStream_t stream);
 int mask_blocks_per_cta(int G, int d, int max_blocks);
 cudaError_t launch_attn(const AttnArgs& a, const AttnLaunch& L, int block, cudaStream_t stream);
 
+// Records a printf-style message for fp_last_error_string() on this thread; returns `code`.
+int set_error(int code, const char* fmt, ...);
+
 }  // namespace fp

@@ -158,6 +158,33 @@ int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void*
                                  const int32_t* kv_cnt, const int32_t* kv_idx, void* out,
                                  float* lse, void* workspace, void* stream);
 
+/*
+ * fp_pool_qk followed by fp_build_block_mask, for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment variant of stages 1 and 2, with the same
+ * arguments and results as those two calls, minus the q_pool / k_pool buffers.
+ *
+ * Who needs it: a serving engine that hands nearly all free HBM to its KV-cache pool at start-up
+ * and must not allocate while serving; code that cannot afford the device synchronisation that
+ * cudaMalloc / cudaFree imply; a host application that passes the library only preallocated
+ * input and output buffers. The pooled means then live in a file-scope device array of this
+ * library, 32 MiB per GPU that loads the library, held until the process exits.
+ *
+ * Limit: (Hq + Hkv) * total_blocks * d <= 8 Mi floats; larger problems return
+ * FP_ERR_INVALID_ARG with a message (use the two regular calls with caller buffers). The first
+ * call on each device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture. All calls share the array
+ * (each call rewrites the pooled values it reads, nothing needs clearing), so calls whose work
+ * overlaps on the same GPU race. No device memory is allocated by this call.
+ */
+int fp_pool_and_mask_noalloc(const void* q, const void* k, int dtype, const float* q_scale,
+                             const float* k_scale, const int32_t* cu_seqlens,
+                             const int32_t* cu_blocks, int batch, int total_tokens,
+                             int total_blocks, int max_blocks, int Hq, int Hkv, int d, int block,
+                             const int32_t* k_page_table, int page_size, int max_pages,
+                             int num_pages, float alpha, float scale, int flags,
+                             uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx,
+                             void* stream);
+
 /* Bytes of device workspace the attention calls need (a fixed small size). */
 size_t fp_workspace_size(void);
 
