@@ -144,7 +144,7 @@ int fp_build_block_mask(const float* q_pool, const float* k_pool, const int32_t*
   if (total_blocks == 0) return FP_OK;
   const int G = Hq / Hkv;
   const int nb = fp::mask_blocks_per_cta(G, d, max_blocks);
-  if (nb == 0)
+  if (nb == 0 && !fp::mask_tc_supported(G, d))
     return fail(FP_ERR_UNSUPPORTED, "%d blocks per request with %d heads per KV head exceed the "
                 "shared-memory score rows of the mask kernel", max_blocks, G);
   fp::MaskArgs a{};

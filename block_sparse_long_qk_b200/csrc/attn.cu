@@ -24,6 +24,8 @@
 // and is consumed by the PV MMA straight from TMEM. All waits are bounded (fp_common.cuh).
 #include <math.h>
 
+#include <type_traits>
+
 #include "fp_common.cuh"
 #include "fp_launch.h"
 
@@ -324,26 +326,89 @@ __global__ void __launch_bounds__(384, 1)
     int n = 0;
     bool ok = true;
     int i = 0;
-    for (;;) {
-      const int J = next_valid(T.list, T.cnt, i, T.I, a.status, r == 0);
-      if (J < 0) break;
+    // P = 2^(s * sl2 - mu) for the whole row, packed and written over the S columns of TMEM;
+    // returns the row sum. Off the diagonal, one column pair in four takes the FMA-pipe
+    // polynomial instead of MUFU ex2, so the exponentials do not outrun the tensor core on
+    // the MUFU unit. Four independent partial sums keep the add chain short.
+    // P = 2^(s * sl2 - mu) for the row, re-read from TMEM 64 columns at a time (so the whole
+    // S row never has to stay in registers), packed and written over the S columns already
+    // read; returns the row sum. Off the diagonal, one column pair in four takes the FMA-pipe
+    // polynomial instead of MUFU ex2, so the exponentials do not outrun the tensor core on the
+    // MUFU unit. Four independent partial sums keep the add chain short.
+    auto p_pass = [&](float mu, auto diag_tag) -> float {
+      constexpr bool diag = decltype(diag_tag)::value;
+      const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-mu, -mu);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int h0 = 0; h0 < BN; h0 += 64) {
+        float sv[64];
+        tmem_ld32(s_tm + h0, sv);
+        if constexpr (BN > 32) tmem_ld32(s_tm + h0 + 32, sv + 32);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c1 = 0; c1 < 64 && h0 + c1 < BN; c1 += 32) {
+          const int c0 = h0 + c1;
+          float2 pp[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float2 x = ffma2(make_float2(sv[c1 + c], sv[c1 + c + 1]), sc2, nm2);
+            if constexpr (diag) {
+              if (c0 + c > r) x.x = -INFINITY;
+              if (c0 + c + 1 > r) x.y = -INFINITY;
+            }
+            pp[c / 2] = (!diag && (c / 2) % 4 == 3) ? exp2_poly2(x)
+                                                     : make_float2(ex2(x.x), ex2(x.y));
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[e % 4] = fadd2(acc[e % 4], pp[e]);
+          if constexpr (FP8) {
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              w[e] = pack_e4m3x4(pp[2 * e].x, pp[2 * e].y, pp[2 * e + 1].x, pp[2 * e + 1].y);
+            tmem_st8(s_tm + c0 / 4, w);
+          } else {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(pp[e].x, pp[e].y);
+            tmem_st16(s_tm + c0 / 2, w);
+          }
+        }
+      }
+      const float2 t = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+      return t.x + t.y;
+    };
+    int J = next_valid(T.list, T.cnt, i, T.I, a.status, r == 0);
+    while (J >= 0) {
+      // The next list entry is fetched before the wait, off the critical path.
+      const int J_next = next_valid(T.list, T.cnt, i, T.I, a.status, r == 0);
       const bool got = !sh.abort_flag && mbar_wait(&sh.s_full[t], n & 1);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN; c += 32) tmem_ld32(s_tm + c, s + c);
-      tmem_ld_wait();
       const bool diag = (J == T.I);
-      if (diag) {  // causal mask inside the diagonal block: key c > query r
+      // Row max over the S row (causal mask inside the diagonal block: key c > query r), read
+      // from TMEM in two halves, as a tree of 8 independent 3-input maxima.
+      float mr[8];
 #pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = (c > r) ? -INFINITY : s[c];
+      for (int e = 0; e < 8; ++e) mr[e] = -INFINITY;
+#pragma unroll
+      for (int h0 = 0; h0 < BN; h0 += 64) {
+        float sv[64];
+        tmem_ld32(s_tm + h0, sv);
+        if constexpr (BN > 32) tmem_ld32(s_tm + h0 + 32, sv + 32);
+        tmem_ld_wait();
+        if (diag) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) sv[c] = (h0 + c > r) ? -INFINITY : sv[c];
+        }
+#pragma unroll
+        for (int c = 0; c < 64 && h0 + c < BN; c += 2)
+          mr[(c / 2) % 8] = fmax3(mr[(c / 2) % 8], sv[c], sv[c + 1]);
       }
-      float mraw = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BN; c += 2) mraw = fmax3(mraw, s[c], s[c + 1]);
-      const float mx = mraw * sl2;  // sl2 > 0: the max commutes with the scaling
-      // Lazy rescaling: keep the stale max unless the row max grew by more than 2^8, so P
+      const float mx = fmax3(fmax3(mr[0], mr[1], mr[2]), fmax3(mr[3], mr[4], mr[5]),
+                             fmaxf(mr[6], mr[7])) * sl2;  // sl2 > 0: max commutes with scaling
+      // Lazy rescaling: keep the stale max m unless the row max grew by more than 2^8, so P
       // stays <= 256 (exact in fp32 accumulation, in range for bf16 and e4m3).
       bool rescale = false;
       float f = 1.f;
@@ -356,43 +421,7 @@ __global__ void __launch_bounds__(384, 1)
         rescale = true;
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
-      const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-mu, -mu);
-      float2 sum2 = make_float2(0.f, 0.f);
-      // P = 2^(s * sl2 - m) in 32-column chunks, packed and written over the S columns of TMEM.
-      // Off the diagonal, one column pair in four takes the FMA-pipe polynomial instead of
-      // MUFU ex2, so the exponentials do not outrun the tensor core on the MUFU unit.
-#pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        float2 pp[16];
-        if (diag) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float2 x = ffma2(make_float2(s[c0 + c], s[c0 + c + 1]), sc2, nm2);
-            pp[c / 2] = make_float2(ex2(x.x), ex2(x.y));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float2 x = ffma2(make_float2(s[c0 + c], s[c0 + c + 1]), sc2, nm2);
-            pp[c / 2] = ((c / 2) % 4 == 3) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) sum2 = fadd2(sum2, pp[e]);
-        if constexpr (FP8) {
-          uint32_t w[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            w[e] = pack_e4m3x4(pp[2 * e].x, pp[2 * e].y, pp[2 * e + 1].x, pp[2 * e + 1].y);
-          tmem_st8(s_tm + c0 / 4, w);
-        } else {
-          uint32_t w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(pp[e].x, pp[e].y);
-          tmem_st16(s_tm + c0 / 2, w);
-        }
-      }
-      const float sum = sum2.x + sum2.y;
+      const float sum = diag ? p_pass(mu, std::true_type{}) : p_pass(mu, std::false_type{});
       l += sum;
       // tcgen05.ld/st are warp-collective: when any row of the warp rescales, the whole warp
       // runs the pass (f = 1 for rows that keep their max).
@@ -414,6 +443,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(&sh.p_full[t]);
       ++n;
+      J = J_next;
     }
     // Epilogue: wait for the last PV of this tile, normalise, store.
     const bool fin = ok && !sh.abort_flag && mbar_wait(&sh.o_final[t], 0);

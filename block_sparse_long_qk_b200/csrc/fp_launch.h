@@ -64,6 +64,8 @@ struct AttnLaunch {
 cudaError_t launch_pool(const PoolArgs& a, bool e4m3, cudaStream_t stream);
 cudaError_t launch_mask(const MaskArgs& a, cudaStream_t stream);
 int mask_blocks_per_cta(int G, int d, int max_blocks);
+bool mask_tc_supported(int G, int d);   // tensor-core scores (mask_tc.cu) apply
+cudaError_t launch_mask_tc(const MaskArgs& a, cudaStream_t stream);
 cudaError_t launch_attn(const AttnArgs& a, const AttnLaunch& L, int block, cudaStream_t stream);
 
 // Records a printf-style message for fp_last_error_string() on this thread; returns `code`.

@@ -177,6 +177,7 @@ int mask_blocks_per_cta(int G, int d, int max_blocks) {
 }
 
 cudaError_t launch_mask(const MaskArgs& in, cudaStream_t stream) {
+  if (mask_tc_supported(in.G, in.d)) return launch_mask_tc(in, stream);
   MaskArgs a = in;
   const size_t smem = mask_smem_bytes(a.G * a.NB, a.d, a.max_blocks);
   cudaError_t e = cudaFuncSetAttribute(mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

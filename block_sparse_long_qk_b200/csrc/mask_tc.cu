@@ -1,0 +1,338 @@
+// Stage 2 on the tensor cores: pooled block scores, max-based threshold, mask and index lists.
+//
+// Same definition as mask.cu ("FlashPrefill: Instantaneous Pattern Discovery and Thresholding
+// for Ultra-Fast Long-Context Prefilling", technical summary 2.B: keep J iff
+// s_J - max_{J'<=I} s_J' >= ln(alpha), plus the forced first and diagonal blocks), but the
+// scores come from tcgen05.mma instead of fp32 FFMA. The threshold compare has to hold to well
+// under 1e-3 in log space, which a single bf16 product does not; each fp32 operand x is split
+// into bf16 x_hi = bf16(x) and x_lo = bf16(x - x_hi) (16 significant bits together), and
+//   q . k ~= q_hi . k_hi + q_hi . k_lo + q_lo . k_hi       (fp32 accumulation in TMEM),
+// which leaves a relative error of about 3 * 2^-18 of sum |q_c k_c| (the dropped q_lo . k_lo and
+// the bf16 rounding of the residuals).
+//
+// One CTA = 128 query rows (the G heads of KV head g times 128/G consecutive query blocks) x
+// every key block its rows need, in chunks of 128 key blocks: S = Q K^T is an M=128, N=128,
+// K=d tile. Pass 0 takes each row's max over its causal, same-request blocks; pass 1 recomputes
+// the chunks and writes the keep bits and the ascending index list. Operands are converted
+// from fp32 and written to shared memory in the 128-byte-swizzled K-major layout by all 256
+// threads, double-buffered against the MMAs; S is double-buffered in TMEM (2 x 128 columns).
+// Warps 0-3 own the 128 TMEM lanes (one query row per thread) for the epilogue.
+#include <math.h>
+
+#include "fp_common.cuh"
+#include "fp_launch.h"
+
+namespace fp {
+
+namespace {
+
+constexpr int kTcThreads = 256;
+constexpr int kTcRows = 128;  // M
+constexpr int kTcKeys = 128;  // N per chunk
+
+template <int D>
+struct TcCfg {
+  static constexpr int kTile = kTcRows * D * 2;      // bytes of one bf16 [128 x D] operand
+  static constexpr int kAHi = 0, kALo = kTile;
+  static constexpr int kB = 2 * kTile;               // B[buf][hi/lo]
+  static constexpr int kMeta = kB + 4 * kTile;
+  static constexpr int kSmem = kMeta + 4 * kTcRows * 4 + 64 + 1024;
+  static constexpr int kKSteps = D / 16;
+};
+
+// Writes 8 consecutive values (columns k0..k0+7, k0 % 8 == 0) of row r of a K-major,
+// 128-byte-swizzled bf16 tile as hi and lo parts.
+__device__ __forceinline__ void put8(uint8_t* hi_tile, uint8_t* lo_tile, int rows, int r, int k0,
+                                     const float* v) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * i]);
+    const __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * i + 1]);
+    const float r0 = v[2 * i] - __bfloat162float(h0);
+    const float r1 = v[2 * i + 1] - __bfloat162float(h1);
+    __nv_bfloat162 hh(h0, h1);
+    h[i] = *reinterpret_cast<uint32_t*>(&hh);
+    l[i] = pack_bf16x2(r0, r1);
+  }
+  const int chunk = k0 / 64, unit = (k0 % 64) / 8;
+  const int off = chunk * rows * 128 + r * 128 + ((unit ^ (r & 7)) << 4);
+  *reinterpret_cast<uint4*>(hi_tile + off) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
+  using C = TcCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  int* row_I = reinterpret_cast<int*>(smem + C::kMeta);  // -1: no row
+  int* row_kb = row_I + kTcRows;
+  int* row_h = row_kb + kTcRows;
+  int* row_g = row_h + kTcRows;
+  uint64_t* done = reinterpret_cast<uint64_t*>(row_g + kTcRows);  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
+
+  const int tid = threadIdx.x, warp = tid / 32;
+  const int g = blockIdx.y;
+  const int rows_blk = kTcRows / a.G;                 // query blocks per CTA
+  // Late query blocks have the longest causal rows: run them first, the short ones fill the tail.
+  const int Ig0 = (gridDim.x - 1 - blockIdx.x) * rows_blk;
+
+  if (tid < kTcRows) {
+    const int Ig = Ig0 + tid / a.G;
+    row_h[tid] = g * a.G + tid % a.G;
+    if (Ig < a.total_blocks) {
+      const int kb = a.cu_blocks ? __ldg(a.cu_blocks + find_request(a.cu_blocks, a.batch, Ig)) : 0;
+      row_I[tid] = Ig - kb;
+      row_kb[tid] = kb;
+      row_g[tid] = Ig;
+    } else {
+      row_I[tid] = -1;
+      row_kb[tid] = 0;
+      row_g[tid] = -1;
+    }
+  }
+  if (tid == 0) {
+    mbar_init(&done[0], 1);
+    mbar_init(&done[1], 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    __syncwarp();
+    tmem_alloc(tmem_slot, 256);
+  }
+
+  // A operand: the 128 rows' pooled queries, split into hi / lo.
+  constexpr int kUnits = D / 8;
+  for (int u = tid; u < kTcRows * kUnits; u += kTcThreads) {
+    const int r = u / kUnits, k0 = (u % kUnits) * 8;
+    const int Ig = Ig0 + r / a.G;
+    float v[8];
+    if (Ig < a.total_blocks) {
+      const float4* src = reinterpret_cast<const float4*>(
+          a.q_pool + (static_cast<size_t>(g * a.G + r % a.G) * a.total_blocks + Ig) * D + k0);
+      const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+      v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+      v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+    put8(smem + C::kAHi, smem + C::kALo, kTcRows, r, k0, v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Key-block range of the CTA: block 0 of its first row's request .. its last row's block.
+  const int last = min(Ig0 + rows_blk, a.total_blocks) - 1;
+  const int Jg_lo = row_kb[0];
+  const int nch = (last - Jg_lo) / kTcKeys + 1;
+  const int W = 2 * nch;  // pass 0 chunks, then pass 1 chunks
+
+  // Each thread owns kPer 8-value units of the chunk; all its loads are issued before any
+  // conversion so that they are in flight together.
+  constexpr int kPer = kTcKeys * kUnits / kTcThreads;
+  auto stage = [&](int w, int buf) {
+    const int Jg0 = Jg_lo + (w % nch) * kTcKeys;
+    uint8_t* bh = smem + C::kB + (2 * buf) * C::kTile;
+    uint8_t* bl = bh + C::kTile;
+    float4 x[kPer][2];
+#pragma unroll
+    for (int p = 0; p < kPer; ++p) {
+      const int u = tid + p * kTcThreads;
+      const int j = u / kUnits, k0 = (u % kUnits) * 8;
+      const int Jg = Jg0 + j;
+      if (Jg <= last) {
+        const float4* src = reinterpret_cast<const float4*>(
+            a.k_pool + (static_cast<size_t>(g) * a.total_blocks + Jg) * D + k0);
+        x[p][0] = __ldg(src);
+        x[p][1] = __ldg(src + 1);
+      } else {
+        x[p][0] = x[p][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < kPer; ++p) {
+      const int u = tid + p * kTcThreads;
+      const float v[8] = {x[p][0].x, x[p][0].y, x[p][0].z, x[p][0].w,
+                          x[p][1].x, x[p][1].y, x[p][1].z, x[p][1].w};
+      put8(bh, bl, kTcKeys, u / kUnits, (u % kUnits) * 8, v);
+    }
+  };
+
+  constexpr uint32_t idesc = make_idesc(1, 1, 0, kTcRows, kTcKeys);
+  const uint32_t sbase = smem_u32(smem);
+  auto issue = [&](int buf) {
+    const uint32_t d_tm = tmem + buf * kTcKeys;
+    const uint32_t bh = sbase + C::kB + (2 * buf) * C::kTile, bl = bh + C::kTile;
+#pragma unroll
+    for (int kk = 0; kk < C::kKSteps; ++kk) {
+      const uint32_t off = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+      const uint64_t ah = make_sdesc(sbase + C::kAHi + off, 16, 1024);
+      const uint64_t al = make_sdesc(sbase + C::kALo + off, 16, 1024);
+      const uint64_t dh = make_sdesc(bh + off, 16, 1024);
+      const uint64_t dl = make_sdesc(bl + off, 16, 1024);
+      mma_f16_ss(d_tm, ah, dh, idesc, kk > 0 ? 1u : 0u);
+      mma_f16_ss(d_tm, ah, dl, idesc, 1u);
+      mma_f16_ss(d_tm, al, dh, idesc, 1u);
+    }
+    tc_commit(&done[buf]);
+  };
+
+  // Row state (warps 0-3, one row per thread).
+  const int r = tid;
+  const bool owner = tid < kTcRows;
+  const int I = owner ? row_I[r] : -1;
+  const int kb = owner ? row_kb[r] : 0;
+  float rmax = -INFINITY;
+  int cnt = 0;
+  const int words = (a.max_blocks + 31) / 32;
+  const size_t row = owner && I >= 0
+                         ? static_cast<size_t>(row_h[r]) * a.total_blocks + row_g[r] : 0;
+  int32_t* idx = a.kv_idx + row * a.max_blocks;
+  uint32_t* bits_row = a.mask_bits ? a.mask_bits + row * words : nullptr;
+  // Keep bits are produced 32 columns at a time starting at an arbitrary J; they are merged
+  // into 32-bit words (pending word `cur_word` with bits `wbits`) and written in order, with
+  // zero words for gaps.
+  int cur_word = 0, next_word = 0;
+  uint32_t wbits = 0;
+  auto emit_word = [&](int w, uint32_t b) {
+    if (!bits_row) return;
+    for (; next_word < w; ++next_word) bits_row[next_word] = 0u;
+    bits_row[w] = b;
+    next_word = w + 1;
+  };
+  auto feed = [&](int Jb, uint32_t km) {  // bit e of km = block Jb + e kept (Jb >= 0)
+    const int w = Jb >> 5, sh = Jb & 31;
+    const uint32_t lo = km << sh, hi = sh ? (km >> (32 - sh)) : 0u;
+    if (w != cur_word) {
+      emit_word(cur_word, wbits);
+      wbits = 0;
+      cur_word = w;
+    }
+    wbits |= lo;
+    if (hi) {
+      emit_word(cur_word, wbits);
+      cur_word = w + 1;
+      wbits = hi;
+    }
+  };
+
+  auto process = [&](int w, int buf) {
+    tc_fence_after();
+    if (warp >= 4) return;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int J0 = Jg_lo + (w % nch) * kTcKeys - kb;  // request-local block of column 0
+    const bool pass0 = w < nch;
+#pragma unroll 1
+    for (int c = 0; c < kTcKeys; c += 32) {
+      float v[32];
+      tmem_ld32(tmem + lane_base + buf * kTcKeys + c, v);
+      tmem_ld_wait();
+      const int Jb = J0 + c;
+      const int lo = max(0, -Jb), hi = min(31, I - Jb);  // valid columns lo..hi
+      if (I < 0 || hi < lo) continue;
+      const uint32_t valid = (hi == 31 ? 0xffffffffu : ((2u << hi) - 1u)) & (~0u << lo);
+      if (pass0) {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if ((valid >> e) & 1u) m4[e % 4] = fmaxf(m4[e % 4], v[e]);
+        rmax = fmaxf(rmax, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale);
+      } else {
+        uint32_t km = 0;
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          km |= (v[e] * a.scale - rmax >= a.log_alpha ? 1u : 0u) << e;
+        if ((a.flags & FP_FORCE_FIRST) && Jb <= 0 && 0 < Jb + 32) km |= 1u << (-Jb);
+        if ((a.flags & FP_FORCE_DIAG) && Jb <= I && I < Jb + 32) km |= 1u << (I - Jb);
+        km &= valid;
+        if (km) {
+          // Columns before the row's request (Jb < 0) are never valid: drop them so the bits
+          // start at J >= 0 (then -Jb <= lo <= 31).
+          int Jn = Jb;
+          if (Jn < 0) {
+            km >>= -Jn;
+            Jn = 0;
+          }
+          feed(Jn, km);
+          for (uint32_t t = km; t; t &= t - 1) idx[cnt++] = Jn + __ffs(t) - 1;
+        }
+      }
+    }
+  };
+
+  stage(0, 0);
+  fence_async_smem();
+  __syncthreads();
+  for (int w = 0; w < W; ++w) {
+    const int b = w & 1;
+    if (tid == 0) {
+      tc_fence_after();
+      issue(b);
+    }
+    if (w >= 1) {
+      // All threads wait for the previous chunk's MMAs: its B buffer is restaged below and its
+      // TMEM columns are read now. The wait is bounded; every thread stays in the loop either
+      // way, so the block barriers below always match.
+      const bool ok = mbar_wait(&done[b ^ 1], ((w - 1) >> 1) & 1);
+      if (__all_sync(0xffffffffu, ok)) process(w - 1, b ^ 1);
+    }
+    if (w + 1 < W) stage(w + 1, b ^ 1);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+  {
+    const bool ok = mbar_wait(&done[(W - 1) & 1], ((W - 1) >> 1) & 1);
+    if (__all_sync(0xffffffffu, ok)) process(W - 1, (W - 1) & 1);
+  }
+
+  if (owner && I >= 0) {
+    emit_word(cur_word, wbits);
+    if (bits_row)
+      for (; next_word < words; ++next_word) bits_row[next_word] = 0u;
+    a.kv_cnt[row] = cnt;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace
+
+bool mask_tc_supported(int G, int d) {
+  return (d == 64 || d == 128) && G >= 1 && G <= kTcRows && kTcRows % G == 0;
+}
+
+cudaError_t launch_mask_tc(const MaskArgs& a, cudaStream_t stream) {
+  const int rows_blk = kTcRows / a.G;
+  dim3 grid((a.total_blocks + rows_blk - 1) / rows_blk, a.Hkv);
+  if (a.d == 128) {
+    cudaError_t e = cudaFuncSetAttribute(mask_tc_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         TcCfg<128>::kSmem);
+    if (e != cudaSuccess) return e;
+    mask_tc_kernel<128><<<grid, kTcThreads, TcCfg<128>::kSmem, stream>>>(a);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(mask_tc_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         TcCfg<64>::kSmem);
+    if (e != cudaSuccess) return e;
+    mask_tc_kernel<64><<<grid, kTcThreads, TcCfg<64>::kSmem, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fp
