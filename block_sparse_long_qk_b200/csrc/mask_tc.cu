@@ -14,9 +14,11 @@
 // every key block its rows need, in chunks of 128 key blocks: S = Q K^T is an M=128, N=128,
 // K=d tile. Pass 0 takes each row's max over its causal, same-request blocks; pass 1 recomputes
 // the chunks and writes the keep bits and the ascending index list. Operands are converted
-// from fp32 and written to shared memory in the 128-byte-swizzled K-major layout by all 256
+// from fp32 and written to shared memory in the 128-byte-swizzled K-major layout by all 512
 // threads, double-buffered against the MMAs; S is double-buffered in TMEM (2 x 128 columns).
-// Warps 0-3 own the 128 TMEM lanes (one query row per thread) for the epilogue.
+// In the epilogue warp w reads TMEM lane quarter w % 4 (32 query rows) and column group w / 4
+// (32 key blocks): four threads share a row, combining their partial maxima once at the pass
+// boundary and their kept counts through a per-chunk prefix in shared memory.
 #include <math.h>
 
 #include "fp_common.cuh"
@@ -26,7 +28,7 @@ namespace fp {
 
 namespace {
 
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 512;
 constexpr int kTcRows = 128;  // M
 constexpr int kTcKeys = 128;  // N per chunk
 
@@ -36,7 +38,9 @@ struct TcCfg {
   static constexpr int kAHi = 0, kALo = kTile;
   static constexpr int kB = 2 * kTile;               // B[buf][hi/lo]
   static constexpr int kMeta = kB + 4 * kTile;
-  static constexpr int kSmem = kMeta + 4 * kTcRows * 4 + 64 + 1024;
+  // row metadata (4 x 128 ints), per-chunk kept counts (2 x 4 x 128 ints), partial maxima
+  // (4 x 128 floats), barriers and the TMEM slot, alignment slack
+  static constexpr int kSmem = kMeta + (4 + 8 + 4) * kTcRows * 4 + 64 + 1024;
   static constexpr int kKSteps = D / 16;
 };
 
@@ -47,13 +51,11 @@ __device__ __forceinline__ void put8(uint8_t* hi_tile, uint8_t* lo_tile, int row
   uint32_t h[4], l[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * i]);
-    const __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * i + 1]);
-    const float r0 = v[2 * i] - __bfloat162float(h0);
-    const float r1 = v[2 * i + 1] - __bfloat162float(h1);
-    __nv_bfloat162 hh(h0, h1);
-    h[i] = *reinterpret_cast<uint32_t*>(&hh);
-    l[i] = pack_bf16x2(r0, r1);
+    // Packed conversions (two values per instruction) for the hi part and the residual.
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    const float2 hf = __bfloat1622float2(hh);
+    h[i] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[i] = pack_bf16x2(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
   }
   const int chunk = k0 / 64, unit = (k0 % 64) / 8;
   const int off = chunk * rows * 128 + r * 128 + ((unit ^ (r & 7)) << 4);
@@ -74,7 +76,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
   int* row_kb = row_I + kTcRows;
   int* row_h = row_kb + kTcRows;
   int* row_g = row_h + kTcRows;
-  uint64_t* done = reinterpret_cast<uint64_t*>(row_g + kTcRows);  // [2]
+  int* cnt_part = row_g + kTcRows;                    // [2][4][128] kept counts per column group
+  float* max_part = reinterpret_cast<float*>(cnt_part + 8 * kTcRows);  // [4][128]
+  uint64_t* done = reinterpret_cast<uint64_t*>(max_part + 4 * kTcRows);  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
 
   const int tid = threadIdx.x, warp = tid / 32;
@@ -101,6 +105,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
     mbar_init(&done[0], 1);
     mbar_init(&done[1], 1);
     fence_barrier_init();
+  }
+  // The CTA owns its 128 rows of mask words: zero them, keep bits are OR-ed in later.
+  if (a.mask_bits != nullptr) {
+    const int words = (a.max_blocks + 31) / 32;
+    for (int i = tid; i < kTcRows * words; i += kTcThreads) {
+      const int rr = i / words;
+      const int Ig = Ig0 + rr / a.G;
+      if (Ig < a.total_blocks)
+        a.mask_bits[(static_cast<size_t>(g * a.G + rr % a.G) * a.total_blocks + Ig) * words +
+                    i % words] = 0u;
+    }
   }
   if (warp == 0) {
     __syncwarp();
@@ -136,14 +151,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
   const int nch = (last - Jg_lo) / kTcKeys + 1;
   const int W = 2 * nch;  // pass 0 chunks, then pass 1 chunks
 
-  // Each thread owns kPer 8-value units of the chunk; all its loads are issued before any
-  // conversion so that they are in flight together.
+  // Each thread owns kPer 8-value units of a chunk. `fetch` issues all of its global loads into
+  // registers (so they are in flight together, and can be in flight while the tensor core
+  // works); `store` converts them and writes the chunk's hi / lo tiles.
   constexpr int kPer = kTcKeys * kUnits / kTcThreads;
-  auto stage = [&](int w, int buf) {
+  float4 xk[kPer][2];
+  auto fetch = [&](int w) {
     const int Jg0 = Jg_lo + (w % nch) * kTcKeys;
-    uint8_t* bh = smem + C::kB + (2 * buf) * C::kTile;
-    uint8_t* bl = bh + C::kTile;
-    float4 x[kPer][2];
 #pragma unroll
     for (int p = 0; p < kPer; ++p) {
       const int u = tid + p * kTcThreads;
@@ -152,17 +166,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
       if (Jg <= last) {
         const float4* src = reinterpret_cast<const float4*>(
             a.k_pool + (static_cast<size_t>(g) * a.total_blocks + Jg) * D + k0);
-        x[p][0] = __ldg(src);
-        x[p][1] = __ldg(src + 1);
+        xk[p][0] = __ldg(src);
+        xk[p][1] = __ldg(src + 1);
       } else {
-        x[p][0] = x[p][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        xk[p][0] = xk[p][1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+  };
+  auto store = [&](int buf) {
+    uint8_t* bh = smem + C::kB + (2 * buf) * C::kTile;
+    uint8_t* bl = bh + C::kTile;
 #pragma unroll
     for (int p = 0; p < kPer; ++p) {
       const int u = tid + p * kTcThreads;
-      const float v[8] = {x[p][0].x, x[p][0].y, x[p][0].z, x[p][0].w,
-                          x[p][1].x, x[p][1].y, x[p][1].z, x[p][1].w};
+      const float v[8] = {xk[p][0].x, xk[p][0].y, xk[p][0].z, xk[p][0].w,
+                          xk[p][1].x, xk[p][1].y, xk[p][1].z, xk[p][1].w};
       put8(bh, bl, kTcKeys, u / kUnits, (u % kUnits) * 8, v);
     }
   };
@@ -186,90 +204,100 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
     tc_commit(&done[buf]);
   };
 
-  // Row state (warps 0-3, one row per thread).
-  const int r = tid;
-  const bool owner = tid < kTcRows;
-  const int I = owner ? row_I[r] : -1;
-  const int kb = owner ? row_kb[r] : 0;
+  // Epilogue state: thread (quarter, column group) owns query row r and 32 of the 128 columns
+  // of each chunk.
+  const int quarter = warp & 3, cgrp = warp >> 2;
+  const int r = quarter * 32 + (tid & 31);
+  const int I = row_I[r];
+  const int kb = row_kb[r];
   float rmax = -INFINITY;
-  int cnt = 0;
+  int cnt = 0;                     // kept blocks of the row so far (same in all 4 threads)
+  uint32_t pend_km = 0;            // keep bits of the previous chunk, written one chunk later
+  int pend_J = 0, pend_item = -1;
   const int words = (a.max_blocks + 31) / 32;
-  const size_t row = owner && I >= 0
-                         ? static_cast<size_t>(row_h[r]) * a.total_blocks + row_g[r] : 0;
+  const size_t row = I >= 0 ? static_cast<size_t>(row_h[r]) * a.total_blocks + row_g[r] : 0;
   int32_t* idx = a.kv_idx + row * a.max_blocks;
   uint32_t* bits_row = a.mask_bits ? a.mask_bits + row * words : nullptr;
-  // Keep bits are produced 32 columns at a time starting at an arbitrary J; they are merged
-  // into 32-bit words (pending word `cur_word` with bits `wbits`) and written in order, with
-  // zero words for gaps.
-  int cur_word = 0, next_word = 0;
-  uint32_t wbits = 0;
-  auto emit_word = [&](int w, uint32_t b) {
-    if (!bits_row) return;
-    for (; next_word < w; ++next_word) bits_row[next_word] = 0u;
-    bits_row[w] = b;
-    next_word = w + 1;
-  };
-  auto feed = [&](int Jb, uint32_t km) {  // bit e of km = block Jb + e kept (Jb >= 0)
-    const int w = Jb >> 5, sh = Jb & 31;
-    const uint32_t lo = km << sh, hi = sh ? (km >> (32 - sh)) : 0u;
-    if (w != cur_word) {
-      emit_word(cur_word, wbits);
-      wbits = 0;
-      cur_word = w;
+
+  // Writes the previous chunk's kept indices at their place in the ascending list, using the
+  // kept counts of the four column groups of that chunk (visible after the block barrier).
+  auto flush = [&]() {
+    if (pend_item < 0) return;
+    const int* cp = cnt_part + (pend_item & 1) * 4 * kTcRows;
+    int before = 0, total = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = cp[q * kTcRows + r];
+      before += q < cgrp ? c : 0;
+      total += c;
     }
-    wbits |= lo;
-    if (hi) {
-      emit_word(cur_word, wbits);
-      cur_word = w + 1;
-      wbits = hi;
+    if (pend_km) {
+      int o = cnt + before;
+      for (uint32_t t = pend_km; t; t &= t - 1) idx[o++] = pend_J + __ffs(t) - 1;
+      if (bits_row) {
+        const int w0 = pend_J >> 5, sh = pend_J & 31;
+        atomicOr(bits_row + w0, pend_km << sh);
+        if (sh && (pend_km >> (32 - sh))) atomicOr(bits_row + w0 + 1, pend_km >> (32 - sh));
+      }
     }
+    cnt += total;
+    pend_item = -1;
   };
 
   auto process = [&](int w, int buf) {
     tc_fence_after();
-    if (warp >= 4) return;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int J0 = Jg_lo + (w % nch) * kTcKeys - kb;  // request-local block of column 0
+    float v[32];
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    tmem_ld32(tmem + lane_base + buf * kTcKeys + cgrp * 32, v);
+    tmem_ld_wait();
+    flush();
     const bool pass0 = w < nch;
-#pragma unroll 1
-    for (int c = 0; c < kTcKeys; c += 32) {
-      float v[32];
-      tmem_ld32(tmem + lane_base + buf * kTcKeys + c, v);
-      tmem_ld_wait();
-      const int Jb = J0 + c;
-      const int lo = max(0, -Jb), hi = min(31, I - Jb);  // valid columns lo..hi
-      if (I < 0 || hi < lo) continue;
-      const uint32_t valid = (hi == 31 ? 0xffffffffu : ((2u << hi) - 1u)) & (~0u << lo);
-      if (pass0) {
+    if (w == nch) {  // first pass-1 chunk: the four partial maxima of pass 0 are in smem
+      rmax = fmaxf(fmaxf(max_part[r], max_part[kTcRows + r]),
+                   fmaxf(max_part[2 * kTcRows + r], max_part[3 * kTcRows + r]));
+    }
+    const int Jb = Jg_lo + (w % nch) * kTcKeys - kb + cgrp * 32;  // request-local J of v[0]
+    const int lo = max(0, -Jb), hi = min(31, I - Jb);            // valid columns lo..hi
+    const bool any = I >= 0 && hi >= lo;
+    const uint32_t valid =
+        any ? ((hi == 31 ? 0xffffffffu : ((2u << hi) - 1u)) & (~0u << lo)) : 0u;
+    if (pass0) {
+      if (any) {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if ((valid >> e) & 1u) m4[e % 4] = fmaxf(m4[e % 4], v[e]);
+        for (int e = 0; e < 32; e += 2)
+          m4[(e / 2) % 4] = fmax3(m4[(e / 2) % 4], ((valid >> e) & 1u) ? v[e] : -INFINITY,
+                                  ((valid >> (e + 1)) & 1u) ? v[e + 1] : -INFINITY);
         rmax = fmaxf(rmax, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale);
-      } else {
-        uint32_t km = 0;
+      }
+      if (w == nch - 1) max_part[cgrp * kTcRows + r] = rmax;
+    } else {
+      uint32_t km = 0;
+      if (any) {
+        // s * scale - max >= ln(alpha)  <=>  s >= (max + ln(alpha)) / scale   (scale > 0)
+        const float thr = (rmax + a.log_alpha) / a.scale;
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          km |= (v[e] * a.scale - rmax >= a.log_alpha ? 1u : 0u) << e;
+        for (int e = 0; e < 32; ++e) km |= (v[e] >= thr ? 1u : 0u) << e;
         if ((a.flags & FP_FORCE_FIRST) && Jb <= 0 && 0 < Jb + 32) km |= 1u << (-Jb);
         if ((a.flags & FP_FORCE_DIAG) && Jb <= I && I < Jb + 32) km |= 1u << (I - Jb);
         km &= valid;
-        if (km) {
-          // Columns before the row's request (Jb < 0) are never valid: drop them so the bits
-          // start at J >= 0 (then -Jb <= lo <= 31).
-          int Jn = Jb;
-          if (Jn < 0) {
-            km >>= -Jn;
-            Jn = 0;
-          }
-          feed(Jn, km);
-          for (uint32_t t = km; t; t &= t - 1) idx[cnt++] = Jn + __ffs(t) - 1;
-        }
       }
+      // Columns before the row's request (Jb < 0) are never valid: drop them so the bits
+      // start at J >= 0 (then -Jb <= lo <= 31).
+      int Jn = Jb;
+      if (km && Jn < 0) {
+        km >>= -Jn;
+        Jn = 0;
+      }
+      cnt_part[(w & 1) * 4 * kTcRows + cgrp * kTcRows + r] = __popc(km);
+      pend_km = km;
+      pend_J = Jn;
+      pend_item = w;
     }
   };
 
-  stage(0, 0);
+  fetch(0);
+  store(0);
   fence_async_smem();
   __syncthreads();
   for (int w = 0; w < W; ++w) {
@@ -278,14 +306,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
       tc_fence_after();
       issue(b);
     }
+    if (w + 1 < W) fetch(w + 1);  // loads in flight while the MMAs of chunk w run
     if (w >= 1) {
-      // All threads wait for the previous chunk's MMAs: its B buffer is restaged below and its
-      // TMEM columns are read now. The wait is bounded; every thread stays in the loop either
-      // way, so the block barriers below always match.
+      // All threads wait for the previous chunk's MMAs: its B buffer is rewritten below and
+      // its TMEM columns are read now. The wait is bounded; every thread stays in the loop
+      // either way, so the block barriers below always match.
       const bool ok = mbar_wait(&done[b ^ 1], ((w - 1) >> 1) & 1);
       if (__all_sync(0xffffffffu, ok)) process(w - 1, b ^ 1);
     }
-    if (w + 1 < W) stage(w + 1, b ^ 1);
+    if (w + 1 < W) store(b ^ 1);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -295,12 +324,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
     if (__all_sync(0xffffffffu, ok)) process(W - 1, (W - 1) & 1);
   }
 
-  if (owner && I >= 0) {
-    emit_word(cur_word, wbits);
-    if (bits_row)
-      for (; next_word < words; ++next_word) bits_row[next_word] = 0u;
-    a.kv_cnt[row] = cnt;
-  }
+  __syncthreads();  // the last chunk's kept counts are visible
+  flush();
+  if (I >= 0 && cgrp == 0) a.kv_cnt[row] = cnt;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

@@ -46,24 +46,26 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
 #pragma unroll
   for (int i = 0; i < EPT; ++i) acc[i] = 0.f;
 
-  // Token row r of the block; nullptr for a paged token whose page entry is out of range.
-  auto row_ptr = [&](int r) -> const int4* {
+  // Row base of token r0 of the block (r0 % 8 == 0; with page_size % 16 == 0 the 8 rows
+  // r0..r0+7 lie in one page, so one page-table lookup serves them); nullptr for a paged
+  // token whose page entry is out of range.
+  auto group_base = [&](int r0) -> const uint8_t* {
     size_t row;
     if (paged) {
-      const int tl = t0 + r;
+      const int tl = t0 + r0;
       const int lp = tl / a.page_size;
       if (lp >= a.max_pages) return nullptr;
       const int page = __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp);
       if (page < 0 || page >= a.num_pages) return nullptr;
       row = static_cast<size_t>(page) * a.page_size + (tl % a.page_size);
     } else {
-      row = static_cast<size_t>(base) + t0 + r;
+      row = static_cast<size_t>(base) + t0 + r0;
     }
-    return reinterpret_cast<const int4*>(src + row * row_bytes + col_bytes);
+    return src + row * row_bytes + col_bytes;
   };
-  auto load = [&](int r) -> int4 {
-    const int4* p = row_ptr(r);
-    return p ? __ldcs(p) : make_int4(0, 0, 0, 0);
+  auto load = [&](const uint8_t* gbase, int u) -> int4 {
+    return gbase ? __ldcs(reinterpret_cast<const int4*>(gbase + u * row_bytes))
+                 : make_int4(0, 0, 0, 0);
   };
 
   auto accumulate = [&](int4 v) {
@@ -89,13 +91,17 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
 
   int r = 0;
   for (; r + 8 <= n; r += 8) {
+    const uint8_t* gbase = group_base(r);
     int4 v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = load(r + u);
+    for (int u = 0; u < 8; ++u) v[u] = load(gbase, u);
 #pragma unroll
     for (int u = 0; u < 8; ++u) accumulate(v[u]);
   }
-  for (; r < n; ++r) accumulate(load(r));
+  if (r < n) {
+    const uint8_t* gbase = group_base(r);
+    for (int u = 0; r + u < n; ++u) accumulate(load(gbase, u));
+  }
 
   const int h = col / a.d;
   const int c = col % a.d;
