@@ -103,6 +103,8 @@ class Layer:
                                     inp.page_table.to(dev))
             self.k = self.v = None
         self.batch = fp.Batch.make(w.seqlens, w.block, dev)
+        self.k_split = torch.empty(fp.k_split_shape(w.Hkv, self.batch.total_blocks, w.d),
+                                   dtype=torch.bfloat16, device=dev)
         self.stream = torch.cuda.current_stream(dev)
         self.ev = []
 
@@ -113,11 +115,11 @@ class Layer:
         if e is not None:
             e[0].record(self.stream)
         qp, kp = fp.pool_qk(self.q, self.k, w.block, batch=b, q_scale=sc["q_scale"],
-                            k_scale=sc["k_scale"], paged=self.paged)
+                            k_scale=sc["k_scale"], paged=self.paged, k_split_out=self.k_split)
         if e is not None:
             e[1].record(self.stream)
         _, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b,
-                                          mask_bits=False)
+                                          mask_bits=False, k_split=self.k_split)
         if e is not None:
             e[2].record(self.stream)
         if self.paged is not None:
@@ -158,7 +160,10 @@ def pool_mask_bytes(w):
     eb = 1 if w.dtype == "e4m3" else 2
     T = w.total_tokens
     nblk = sum((L + w.block - 1) // w.block for L in w.seqlens)
-    return T * (w.Hq + w.Hkv) * w.d * eb + 2 * nblk * (w.Hq + w.Hkv) * w.d * 4
+    # Q and K read once; pooled means written (fp32) and read back by the mask kernel, plus the
+    # bf16 hi / lo split of the pooled keys written and read
+    return (T * (w.Hq + w.Hkv) * w.d * eb + 2 * nblk * (w.Hq + w.Hkv) * w.d * 4
+            + 2 * nblk * w.Hkv * w.d * 4)
 
 
 def cpu_baseline(inp, rows_sample=32, seed=5):

@@ -29,7 +29,7 @@ import torch
 __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_attn",
            "sparse_prefill_attn_paged", "sparse_prefill", "check_status", "workspace",
            "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "header_symbols",
-           "pool_and_mask_noalloc"]
+           "pool_and_mask_noalloc", "k_split_shape"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfpsparse.so")
@@ -47,9 +47,9 @@ _SIGNATURES = {
     "fp_last_error_string": (ctypes.c_char_p, []),
     "fp_workspace_size": (_sz, []),
     "fp_pool_qk": (_i, [_p, _p, _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i,
-                        _i, _p, _p, _p]),
-    "fp_build_block_mask": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _f, _i, _p, _p, _p,
-                                 _p]),
+                        _i, _p, _p, _p, _p]),
+    "fp_build_block_mask": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _f, _i, _p, _p,
+                                 _p, _p]),
     "fp_sparse_prefill_attn": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i,
                                     _i, _i, _i, _f, _p, _p, _p, _p, _p, _p]),
     "fp_sparse_prefill_attn_paged": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _i, _i, _i, _i,
@@ -194,9 +194,11 @@ def _batch_for(q, block, batch):
 
 
 def pool_qk(q, k, block=128, *, batch: Batch | None = None, q_scale=None, k_scale=None,
-            paged: PagedKV | None = None):
+            paged: PagedKV | None = None, k_split_out=None):
     """Block means of Q [T,Hq,d] and K [T,Hkv,d] (or the paged K cache) -> float32
-    q_pool [Hq, nblk, d], k_pool [Hkv, nblk, d]."""
+    q_pool [Hq, nblk, d], k_pool [Hkv, nblk, d]. With ``k_split_out`` (bf16 tensor of
+    ``k_split_shape``) the kernel also writes the hi / lo bf16 split of k_pool there, which
+    ``build_block_mask(k_split=...)`` then loads instead of converting."""
     T, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
     Hkv = kk.shape[-2]
@@ -211,12 +213,17 @@ def pool_qk(q, k, block=128, *, batch: Batch | None = None, q_scale=None, k_scal
         _ptr(q), _ptr(kk), _dtype_code(q), _ptr(q_scale), _ptr(k_scale), cu, cb, b.size, T,
         b.total_blocks, Hq, Hkv, d, block, _ptr(pt), paged.page_size if paged else 0,
         pt.shape[1] if pt is not None else 0, kk.shape[0] if pt is not None else 0,
-        _ptr(q_pool), _ptr(k_pool), _stream(q.device)))
+        _ptr(q_pool), _ptr(k_pool), _ptr(k_split_out), _stream(q.device)))
     return q_pool, k_pool
 
 
+def k_split_shape(Hkv, total_blocks, d):
+    """Shape of the bf16 hi / lo split of the pooled keys: [2, Hkv, total_blocks, d]."""
+    return (2, Hkv, total_blocks, d)
+
+
 def build_block_mask(q_pool, k_pool, alpha=0.1, *, block=128, batch: Batch | None = None,
-                     scale=None, flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True):
+                     scale=None, flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True, k_split=None):
     """Max-based dynamic threshold on the pooled block scores -> (mask_bits or None
     [Hq, nblk, words] uint32 viewed as int32, kv_cnt [Hq, nblk] int32, kv_idx
     [Hq, nblk, max_blocks] int32)."""
@@ -234,7 +241,8 @@ def build_block_mask(q_pool, k_pool, alpha=0.1, *, block=128, batch: Batch | Non
     kv_idx = torch.empty((Hq, nblk, batch.max_blocks), dtype=torch.int32, device=dev)
     cb = _ptr(batch.cu_blocks) if batch.size > 1 else None
     _check(library().fp_build_block_mask(
-        _ptr(q_pool), _ptr(k_pool), cb, batch.size, nblk, batch.max_blocks, Hq, Hkv, d,
+        _ptr(q_pool), _ptr(k_pool), _ptr(k_split), cb, batch.size, nblk, batch.max_blocks, Hq,
+        Hkv, d,
         float(alpha), float(scale), int(flags), _ptr(bits), _ptr(kv_cnt), _ptr(kv_idx),
         _stream(dev)))
     return bits, kv_cnt, kv_idx
@@ -292,9 +300,14 @@ def sparse_prefill(q, k=None, v=None, alpha=0.1, block=128, *, batch: Batch | No
     d = q.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    q_pool, k_pool = pool_qk(q, k, block, batch=b, q_scale=q_scale, k_scale=k_scale, paged=paged)
+    Hkv = (paged.k_cache if paged is not None else k).shape[-2]
+    k_split = torch.empty(k_split_shape(Hkv, b.total_blocks, d), dtype=torch.bfloat16,
+                          device=q.device)
+    q_pool, k_pool = pool_qk(q, k, block, batch=b, q_scale=q_scale, k_scale=k_scale, paged=paged,
+                             k_split_out=k_split)
     _, kv_cnt, kv_idx = build_block_mask(q_pool, k_pool, alpha, block=block, batch=b,
-                                         scale=scale, flags=flags, mask_bits=False)
+                                         scale=scale, flags=flags, mask_bits=False,
+                                         k_split=k_split)
     if paged is not None:
         out, lse = sparse_prefill_attn_paged(q, paged, kv_cnt, kv_idx, b, scale=scale,
                                              q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,

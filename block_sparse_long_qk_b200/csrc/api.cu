@@ -60,6 +60,19 @@ int check_common(int dtype, const float* qs, const float* ks, const float* vs, b
 }  // namespace
 
 namespace fp {
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
 int set_error(int code, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -83,13 +96,14 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
                const float* k_scale, const int32_t* cu_seqlens, const int32_t* cu_blocks,
                int batch, int total_tokens, int total_blocks, int Hq, int Hkv, int d,
                int block, const int32_t* k_page_table, int page_size, int max_pages,
-               int num_pages, float* q_pool, float* k_pool, void* stream) {
+               int num_pages, float* q_pool, float* k_pool, void* k_pool_split, void* stream) {
   g_err.clear();
   int rc = check_common(dtype, q_scale, k_scale, nullptr, false, cu_seqlens, cu_blocks, batch,
                         total_tokens, total_blocks, Hq, Hkv, d, block);
   if (rc) return rc;
   if (!q || !k || !q_pool || !k_pool) return fail(FP_ERR_INVALID_ARG, "null tensor pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool) ||
+      !aligned16(k_pool_split))
     return fail(FP_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   if (k_page_table) {
     if (page_size < 16 || page_size % 16 || block % page_size || max_pages < 1 || num_pages < 1)
@@ -110,6 +124,7 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
   a.page_table = k_page_table;
   a.q_pool = q_pool;
   a.k_pool = k_pool;
+  a.k_split = static_cast<__nv_bfloat16*>(k_pool_split);
   a.batch = batch;
   a.total_tokens = total_tokens;
   a.total_blocks = total_blocks;
@@ -123,10 +138,10 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
   return e == cudaSuccess ? FP_OK : cuda_fail(e, "pool kernel launch");
 }
 
-int fp_build_block_mask(const float* q_pool, const float* k_pool, const int32_t* cu_blocks,
-                        int batch, int total_blocks, int max_blocks, int Hq, int Hkv, int d,
-                        float alpha, float scale, int flags, uint32_t* mask_bits,
-                        int32_t* kv_cnt, int32_t* kv_idx, void* stream) {
+int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_pool_split,
+                        const int32_t* cu_blocks, int batch, int total_blocks, int max_blocks,
+                        int Hq, int Hkv, int d, float alpha, float scale, int flags,
+                        uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* stream) {
   g_err.clear();
   if (!q_pool || !k_pool || !kv_cnt || !kv_idx) return fail(FP_ERR_INVALID_ARG, "null pointer");
   if (batch < 1 || (batch > 1 && !cu_blocks))
@@ -139,7 +154,7 @@ int fp_build_block_mask(const float* q_pool, const float* k_pool, const int32_t*
     return fail(FP_ERR_INVALID_ARG, "bad block counts");
   if (cu_blocks == nullptr && max_blocks != total_blocks)
     return fail(FP_ERR_INVALID_ARG, "one sequence: max_blocks must equal total_blocks");
-  if (!aligned16(q_pool) || !aligned16(k_pool))
+  if (!aligned16(q_pool) || !aligned16(k_pool) || !aligned16(k_pool_split))
     return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
   if (total_blocks == 0) return FP_OK;
   const int G = Hq / Hkv;
@@ -150,6 +165,7 @@ int fp_build_block_mask(const float* q_pool, const float* k_pool, const int32_t*
   fp::MaskArgs a{};
   a.q_pool = q_pool;
   a.k_pool = k_pool;
+  a.k_split = k_pool_split;
   a.cu_blocks = cu_blocks;
   a.mask_bits = mask_bits;
   a.kv_cnt = kv_cnt;

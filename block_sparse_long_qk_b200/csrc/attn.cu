@@ -501,29 +501,10 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // ------------------------------------------------------------------------------------ host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                   CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
 // [rows, heads, d] token-major tensor; box = (one 128-byte chunk of d, 1 head, box_rows rows).
 static bool make_map(CUtensorMap* m, const void* base, bool e4m3, int d, int heads,
                      long long rows, int box_rows) {
-  EncodeTiledFn enc = get_encode_fn();
+  EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const int eb = e4m3 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),

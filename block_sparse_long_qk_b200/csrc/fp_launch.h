@@ -1,6 +1,7 @@
 // Argument structs and host launchers shared by the kernel files and the C ABI (internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -17,6 +18,7 @@ struct PoolArgs {
   const int32_t* page_table;
   float* q_pool;
   float* k_pool;
+  __nv_bfloat16* k_split;  // optional bf16 [2][Hkv][total_blocks][d] hi / lo parts of k_pool
   int batch, total_tokens, total_blocks, Hq, Hkv, d, block, page_size, max_pages, num_pages;
   int q_slices;  // column slices of Q per block (the rest of gridDim.y are K slices)
 };
@@ -24,6 +26,7 @@ struct PoolArgs {
 struct MaskArgs {
   const float* q_pool;
   const float* k_pool;
+  const void* k_split;  // bf16 [2][Hkv][total_blocks][d] hi / lo parts of k_pool, or nullptr
   const int32_t* cu_blocks;
   uint32_t* mask_bits;
   int32_t* kv_cnt;
@@ -67,6 +70,14 @@ int mask_blocks_per_cta(int G, int d, int max_blocks);
 bool mask_tc_supported(int G, int d);   // tensor-core scores (mask_tc.cu) apply
 cudaError_t launch_mask_tc(const MaskArgs& a, cudaStream_t stream);
 cudaError_t launch_attn(const AttnArgs& a, const AttnLaunch& L, int block, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link against libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
 
 // Records a printf-style message for fp_last_error_string() on this thread; returns `code`.
 int set_error(int code, const char* fmt, ...);

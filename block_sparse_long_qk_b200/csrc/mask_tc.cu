@@ -20,6 +20,7 @@
 // (32 key blocks): four threads share a row, combining their partial maxima once at the pass
 // boundary and their kept counts through a per-chunk prefix in shared memory.
 #include <math.h>
+#include <string.h>
 
 #include "fp_common.cuh"
 #include "fp_launch.h"
@@ -41,6 +42,8 @@ struct TcCfg {
   // row metadata (4 x 128 ints), per-chunk kept counts (2 x 4 x 128 ints), partial maxima
   // (4 x 128 floats), barriers and the TMEM slot, alignment slack
   static constexpr int kSmem = kMeta + (4 + 8 + 4) * kTcRows * 4 + 64 + 1024;
+  static constexpr int kBoxBytes = kTcKeys * 128;         // one 128-row x 64-column bf16 box
+  static constexpr int kSplitTx = 2 * (D / 64) * kBoxBytes;  // hi + lo tiles of one chunk
   static constexpr int kKSteps = D / 16;
 };
 
@@ -67,8 +70,12 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
+// kTma: the B operand (pooled keys, split into bf16 hi / lo) is read by TMA from the split that
+// the pool kernel wrote (`tm_split`: 2-D map over [2 * Hkv * total_blocks, d] bf16 with
+// 128-row, 64-column boxes), instead of being converted from fp32 by the threads.
+template <int D, bool kTma>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    mask_tc_kernel(const __grid_constant__ CUtensorMap tm_split, const MaskArgs a) {
   using C = TcCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -79,13 +86,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
   int* cnt_part = row_g + kTcRows;                    // [2][4][128] kept counts per column group
   float* max_part = reinterpret_cast<float*>(cnt_part + 8 * kTcRows);  // [4][128]
   uint64_t* done = reinterpret_cast<uint64_t*>(max_part + 4 * kTcRows);  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 2);
+  uint64_t* full = done + 2;                                              // [2] (TMA)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 2);
 
   const int tid = threadIdx.x, warp = tid / 32;
-  const int g = blockIdx.y;
+  // 1-D grid over (row tile, KV head), ordered so that the late row tiles of every KV head --
+  // the longest causal rows -- launch first and the short ones fill the tail.
+  const int g = blockIdx.x % a.Hkv;
   const int rows_blk = kTcRows / a.G;                 // query blocks per CTA
-  // Late query blocks have the longest causal rows: run them first, the short ones fill the tail.
-  const int Ig0 = (gridDim.x - 1 - blockIdx.x) * rows_blk;
+  const int ntiles = gridDim.x / a.Hkv;
+  const int Ig0 = (ntiles - 1 - static_cast<int>(blockIdx.x) / a.Hkv) * rows_blk;
 
   if (tid < kTcRows) {
     const int Ig = Ig0 + tid / a.G;
@@ -104,7 +114,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
   if (tid == 0) {
     mbar_init(&done[0], 1);
     mbar_init(&done[1], 1);
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
     fence_barrier_init();
+    if constexpr (kTma) prefetch_tensormap(&tm_split);
   }
   // The CTA owns its 128 rows of mask words: zero them, keep bits are OR-ed in later.
   if (a.mask_bits != nullptr) {
@@ -182,6 +195,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
       const float v[8] = {xk[p][0].x, xk[p][0].y, xk[p][0].z, xk[p][0].w,
                           xk[p][1].x, xk[p][1].y, xk[p][1].z, xk[p][1].w};
       put8(bh, bl, kTcKeys, u / kUnits, (u % kUnits) * 8, v);
+    }
+  };
+
+  // One chunk of the B operand by TMA: hi rows g * total_blocks + Jg0 .. +127 and the same rows
+  // of the lo plane (rows past the group's last block carry other data or zeros; their score
+  // columns are never valid).
+  auto tma_chunk = [&](int w, int buf) {
+    const int row = g * a.total_blocks + Jg_lo + (w % nch) * kTcKeys;
+    const int lo_row = a.Hkv * a.total_blocks + row;
+    uint8_t* bh = smem + C::kB + (2 * buf) * C::kTile;
+    uint8_t* bl = bh + C::kTile;
+    mbar_arrive_expect_tx(&full[buf], C::kSplitTx);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_2d(bh + c * C::kBoxBytes, &tm_split, &full[buf], c * 64, row);
+      tma_load_2d(bl + c * C::kBoxBytes, &tm_split, &full[buf], c * 64, lo_row);
     }
   };
 
@@ -296,26 +325,45 @@ __global__ void __launch_bounds__(kTcThreads, 1) mask_tc_kernel(MaskArgs a) {
     }
   };
 
-  fetch(0);
-  store(0);
-  fence_async_smem();
+  if constexpr (kTma) {
+    if (tid == 0) tma_chunk(0, 0);
+  } else {
+    fetch(0);
+    store(0);
+    fence_async_smem();
+  }
   __syncthreads();
   for (int w = 0; w < W; ++w) {
     const int b = w & 1;
-    if (tid == 0) {
-      tc_fence_after();
-      issue(b);
+    if constexpr (kTma) {
+      if (tid == 0) {
+        // chunk w has landed -> its MMAs; then, once chunk w-1's MMAs are done with the
+        // other buffer, start loading chunk w+1 into it.
+        const bool ok_full = mbar_wait(&full[b], (w >> 1) & 1);
+        tc_fence_after();
+        if (ok_full) issue(b);
+        else tc_commit(&done[b]);
+        if (w + 1 < W && (w == 0 || mbar_wait(&done[b ^ 1], ((w - 1) >> 1) & 1)))
+          tma_chunk(w + 1, b ^ 1);
+      }
+    } else {
+      if (tid == 0) {
+        tc_fence_after();
+        issue(b);
+      }
+      if (w + 1 < W) fetch(w + 1);  // loads in flight while the MMAs of chunk w run
     }
-    if (w + 1 < W) fetch(w + 1);  // loads in flight while the MMAs of chunk w run
     if (w >= 1) {
-      // All threads wait for the previous chunk's MMAs: its B buffer is rewritten below and
-      // its TMEM columns are read now. The wait is bounded; every thread stays in the loop
+      // All threads wait for the previous chunk's MMAs: its B buffer is rewritten and its
+      // TMEM columns are read now. The wait is bounded; every thread stays in the loop
       // either way, so the block barriers below always match.
       const bool ok = mbar_wait(&done[b ^ 1], ((w - 1) >> 1) & 1);
       if (__all_sync(0xffffffffu, ok)) process(w - 1, b ^ 1);
     }
-    if (w + 1 < W) store(b ^ 1);
-    fence_async_smem();
+    if constexpr (!kTma) {
+      if (w + 1 < W) store(b ^ 1);
+      fence_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
   }
@@ -342,23 +390,39 @@ bool mask_tc_supported(int G, int d) {
   return (d == 64 || d == 128) && G >= 1 && G <= kTcRows && kTcRows % G == 0;
 }
 
+template <int D, bool kTma>
+static cudaError_t launch_tc(const MaskArgs& a, const CUtensorMap& map, dim3 grid,
+                             cudaStream_t stream) {
+  auto kern = mask_tc_kernel<D, kTma>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       TcCfg<D>::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kTcThreads, TcCfg<D>::kSmem, stream>>>(map, a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mask_tc(const MaskArgs& a, cudaStream_t stream) {
   const int rows_blk = kTcRows / a.G;
-  dim3 grid((a.total_blocks + rows_blk - 1) / rows_blk, a.Hkv);
-  if (a.d == 128) {
-    cudaError_t e = cudaFuncSetAttribute(mask_tc_kernel<128>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TcCfg<128>::kSmem);
-    if (e != cudaSuccess) return e;
-    mask_tc_kernel<128><<<grid, kTcThreads, TcCfg<128>::kSmem, stream>>>(a);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(mask_tc_kernel<64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TcCfg<64>::kSmem);
-    if (e != cudaSuccess) return e;
-    mask_tc_kernel<64><<<grid, kTcThreads, TcCfg<64>::kSmem, stream>>>(a);
+  dim3 grid(((a.total_blocks + rows_blk - 1) / rows_blk) * a.Hkv);
+  CUtensorMap map;
+  memset(&map, 0, sizeof(map));
+  if (a.k_split != nullptr) {
+    EncodeTiledFn enc = tensor_map_encoder();
+    if (enc == nullptr) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.d),
+                          2ull * static_cast<cuuint64_t>(a.Hkv) * a.total_blocks};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.d) * 2};
+    cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(kTcKeys)};
+    cuuint32_t estr[2] = {1u, 1u};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.k_split), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    return a.d == 128 ? launch_tc<128, true>(a, map, grid, stream)
+                      : launch_tc<64, true>(a, map, grid, stream);
   }
-  return cudaGetLastError();
+  return a.d == 128 ? launch_tc<128, false>(a, map, grid, stream)
+                    : launch_tc<64, false>(a, map, grid, stream);
 }
 
 }  // namespace fp

@@ -76,8 +76,8 @@ extern "C" int fp_pool_and_mask_noalloc(
   float* k_pool = scratch + static_cast<size_t>(Hq) * total_blocks * d;
   int rc = fp_pool_qk(q, k, dtype, q_scale, k_scale, cu_seqlens, cu_blocks, batch, total_tokens,
                       total_blocks, Hq, Hkv, d, block, k_page_table, page_size, max_pages,
-                      num_pages, q_pool, k_pool, stream);
+                      num_pages, q_pool, k_pool, nullptr, stream);
   if (rc != FP_OK) return rc;
-  return fp_build_block_mask(q_pool, k_pool, cu_blocks, batch, total_blocks, max_blocks, Hq, Hkv,
-                             d, alpha, scale, flags, mask_bits, kv_cnt, kv_idx, stream);
+  return fp_build_block_mask(q_pool, k_pool, nullptr, cu_blocks, batch, total_blocks, max_blocks,
+                             Hq, Hkv, d, alpha, scale, flags, mask_bits, kv_cnt, kv_idx, stream);
 }

@@ -111,9 +111,28 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
   float* dst = (is_q ? a.q_pool : a.k_pool) +
                (static_cast<size_t>(h) * a.total_blocks + gb) * a.d + c;
 #pragma unroll
+  for (int i = 0; i < EPT; ++i) acc[i] *= s;
+#pragma unroll
   for (int i = 0; i < EPT; i += 4)
-    *reinterpret_cast<float4*>(dst + i) =
-        make_float4(acc[i] * s, acc[i + 1] * s, acc[i + 2] * s, acc[i + 3] * s);
+    *reinterpret_cast<float4*>(dst + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+  if (!is_q && a.k_split != nullptr) {
+    // bf16 hi / lo split of the pooled key (the tensor-core operands of the mask kernel).
+    const size_t plane = static_cast<size_t>(a.Hkv) * a.total_blocks * a.d;
+    __nv_bfloat16* hi = a.k_split + (static_cast<size_t>(h) * a.total_blocks + gb) * a.d + c;
+#pragma unroll
+    for (int i = 0; i < EPT; i += 8) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 hh = __floats2bfloat162_rn(acc[i + 2 * j], acc[i + 2 * j + 1]);
+        const float2 hf = __bfloat1622float2(hh);
+        hw[j] = *reinterpret_cast<const uint32_t*>(&hh);
+        lw[j] = pack_bf16x2(acc[i + 2 * j] - hf.x, acc[i + 2 * j + 1] - hf.y);
+      }
+      *reinterpret_cast<uint4*>(hi + i) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(hi + plane + i) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+  }
 }
 
 cudaError_t launch_pool(const PoolArgs& in, bool e4m3, cudaStream_t stream) {

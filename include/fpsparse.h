@@ -78,6 +78,9 @@ const char* fp_last_error_string(void);
  *            as zeros).
  * q_pool     float32 [Hq, total_blocks, d] (written)
  * k_pool     float32 [Hkv, total_blocks, d] (written)
+ * k_pool_split  NULL, or bf16 [2, Hkv, total_blocks, d] (written): hi = bf16(k_pool) and
+ *            lo = bf16(k_pool - hi), the operand split fp_build_block_mask feeds to the tensor
+ *            cores; passing it on to fp_build_block_mask saves that call the conversion.
  * Supported: d in {64, 128}; block in {64, 128}; Hq % Hkv == 0; page_size a multiple of 16
  * that divides block. Q and K must be 16-byte aligned.
  */
@@ -85,7 +88,7 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
                const float* k_scale, const int32_t* cu_seqlens, const int32_t* cu_blocks,
                int batch, int total_tokens, int total_blocks, int Hq, int Hkv, int d,
                int block, const int32_t* k_page_table, int page_size, int max_pages,
-               int num_pages, float* q_pool, float* k_pool, void* stream);
+               int num_pages, float* q_pool, float* k_pool, void* k_pool_split, void* stream);
 
 /*
  * Stage 2: pooled block scores and the max-based dynamic threshold ("FlashPrefill:
@@ -99,6 +102,8 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
  *           or (flags & FP_FORCE_FIRST and J == 0) or (flags & FP_FORCE_DIAG and J == I).
  * alpha in [0, 1]; alpha = 0 keeps every causal block.
  *
+ * k_pool_split  NULL, or the split written by fp_pool_qk for this k_pool (results are
+ *            identical either way; with it the scores' operands are loaded, not converted)
  * mask_bits  uint32 [Hq, total_blocks, words], words = ceil(max_blocks / 32): bit J % 32 of
  *            word J / 32 is set iff block J is kept (bits above I are 0). May be NULL.
  * kv_cnt     int32 [Hq, total_blocks]: number of kept blocks of the row
@@ -106,10 +111,10 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
  *            ascending order in the first kv_cnt entries (the rest is left untouched)
  * max_blocks largest per-request block count (host int)
  */
-int fp_build_block_mask(const float* q_pool, const float* k_pool, const int32_t* cu_blocks,
-                        int batch, int total_blocks, int max_blocks, int Hq, int Hkv, int d,
-                        float alpha, float scale, int flags, uint32_t* mask_bits,
-                        int32_t* kv_cnt, int32_t* kv_idx, void* stream);
+int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_pool_split,
+                        const int32_t* cu_blocks, int batch, int total_blocks, int max_blocks,
+                        int Hq, int Hkv, int d, float alpha, float scale, int flags,
+                        uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* stream);
 
 /*
  * Stage 3: causal attention over the kept KV blocks only ("FlashPrefill: Instantaneous

@@ -53,7 +53,7 @@ def test_attention_rejects_bad_arguments(over, code):
 
 def test_mask_rejects_alpha_out_of_range():
     lib = fp.library()
-    rc = lib.fp_build_block_mask(16, 16, None, 1, 4, 4, 8, 2, 128, 1.5, 0.1, 3, None, 16, 16,
-                                 None)
+    rc = lib.fp_build_block_mask(16, 16, None, None, 1, 4, 4, 8, 2, 128, 1.5, 0.1, 3, None, 16,
+                                 16, None)
     assert rc == -1
     assert b"alpha" in lib.fp_last_error_string()

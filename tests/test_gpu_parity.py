@@ -94,6 +94,19 @@ def test_pool_and_mask_match_oracle(name, cuda_device):
     lk = lists_to_keeps(cnt, idx, run)
     for a_, b_ in zip(gk, lk):
         assert np.array_equal(a_, b_)
+    # with the pool kernel's hi / lo split of k_pool (TMA-fed mask kernel) the results are the
+    # same bits and lists
+    split = torch.empty(fp.k_split_shape(inp.workload.Hkv, b.total_blocks, inp.workload.d),
+                        dtype=torch.bfloat16, device=cuda_device)
+    qp2, kp2 = fp.pool_qk(q, k, inp.workload.block, batch=b, q_scale=sc["q_scale"],
+                          k_scale=sc["k_scale"], paged=_paged(inp, cuda_device), k_split_out=split)
+    bits2, cnt2, idx2 = fp.build_block_mask(qp2, kp2, alpha, block=inp.workload.block, batch=b,
+                                            k_split=split)
+    torch.cuda.synchronize()
+    assert torch.equal(qp2, qp) and torch.equal(kp2, kp)
+    assert torch.equal(bits2, bits) and torch.equal(cnt2, cnt)
+    for a_, b_ in zip(lk, lists_to_keeps(cnt2, idx2, run)):
+        assert np.array_equal(a_, b_)
 
 
 @pytest.mark.parametrize("name", SMALL)
