@@ -288,9 +288,10 @@ def run_native(args, world, rank, local):
     fp.check_status(dev)
     total_ms = t_start.elapsed_time(t_end)
     ms_step = max_over_ranks(total_ms / args.steps, world, dev)
-    pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    mask_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    pool_l = [e[0].elapsed_time(e[1]) for e in evs]
+    mask_l = [e[1].elapsed_time(e[2]) for e in evs]
+    attn_l = [e[2].elapsed_time(e[3]) for e in evs]
+    pool_ms, mask_ms, attn_ms = (statistics.mean(x) for x in (pool_l, mask_l, attn_l))
 
     alg, executed, density = work_counts(w, cnt, idx, layer.batch)
     pm_bytes = pool_mask_bytes(w)
@@ -328,6 +329,9 @@ def run_native(args, world, rank, local):
             "config": _config(w, args),
             "stages_ms": {"pool": round(pool_ms, 4), "mask": round(mask_ms, 4),
                           "attn": round(attn_ms, 4)},
+            "stages_ms_median_max": {n: [round(statistics.median(x), 4), round(max(x), 4)]
+                                     for n, x in (("pool", pool_l), ("mask", mask_l),
+                                                  ("attn", attn_l))},
             "pool_mask": {"bytes": pm_bytes,
                           "gbs": round(pm_bytes / ((pool_ms + mask_ms) * 1e-3) / 1e9, 1),
                           "frac_hbm": round(pm_bytes / ((pool_ms + mask_ms) * 1e-3) / 1e9 /

@@ -46,6 +46,8 @@ struct AttnCfg {
   static constexpr int kVOff = kKOff + kKSt * kKVBytes;
   static constexpr int kBarOff = kVOff + kVSt * kKVBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+  static_assert(kKSt <= 4 && kVSt <= 4, "ring depth");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
   static constexpr int kTmemUsed = 2 * BN + 2 * D;          // S0 S1 O0 O1
   static constexpr int kTmemCols = kTmemUsed <= 256 ? 256 : 512;  // power-of-2 allocation
   static constexpr uint32_t kS0 = 0, kS1 = BN, kO0 = 2 * BN, kO1 = 2 * BN + D;
@@ -60,7 +62,7 @@ struct Tile {
 
 struct Shared {  // placed at kBarOff
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];  // ring slots (kKSt, kVSt <= 4)
   uint64_t s_full[2], p_full[2], o_final[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -165,9 +167,15 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&sh.q_full, 1);
+    for (int i = 0; i < C::kKSt; ++i) {
+      mbar_init(&sh.k_full[i], 1);
+      mbar_init(&sh.k_empty[i], 1);
+    }
+    for (int i = 0; i < C::kVSt; ++i) {
+      mbar_init(&sh.v_full[i], 1);
+      mbar_init(&sh.v_empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.k_full[i], 1); mbar_init(&sh.k_empty[i], 1);
-      mbar_init(&sh.v_full[i], 1); mbar_init(&sh.v_empty[i], 1);
       mbar_init(&sh.s_full[i], 1); mbar_init(&sh.p_full[i], 128); mbar_init(&sh.o_final[i], 1);
     }
     mbar_init(&sh.drain, 1);
