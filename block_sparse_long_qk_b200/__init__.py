@@ -56,6 +56,7 @@ _SIGNATURES = {
                                           _i, _i, _i, _i, _p, _i, _i, _i, _f, _p, _p, _p, _p,
                                           _p, _p]),
     "fp_check_status": (_i, [_p, _p]),
+    "fp_debug_skip_k_load": (_i, [_i]),
     "fp_pool_and_mask_noalloc": (_i, [_p, _p, _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
                                       _i, _p, _i, _i, _i, _f, _f, _i, _p, _p, _p, _p]),
 }

@@ -12,6 +12,7 @@
 namespace {
 
 thread_local std::string g_err;
+thread_local int g_fault_skip_k = -1;  // one-shot test hook for the next attention call
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -240,6 +241,8 @@ static int attn_common(const void* q, const void* k, const void* v, int dtype,
   a.pair_heads = (G % 2 == 0) ? 1 : 0;
   a.num_items = a.pair_heads ? (Hq / 2) * total_blocks : Hq * total_blocks;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.fault_skip_k = g_fault_skip_k;
+  g_fault_skip_k = -1;
   fp::AttnLaunch L{};
   L.q = q;
   L.k = k;
@@ -284,6 +287,13 @@ int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void*
                      cu_blocks, batch, total_tokens, total_blocks, max_blocks, Hq, Hkv, d,
                      block, page_table, page_size, max_pages, num_pages, scale, kv_cnt, kv_idx,
                      out, lse, workspace, stream);
+}
+
+int fp_debug_skip_k_load(int union_block) {
+  g_err.clear();
+  if (union_block < 0) return fail(FP_ERR_INVALID_ARG, "union block index must be >= 0");
+  g_fault_skip_k = union_block;
+  return FP_OK;
 }
 
 int fp_check_status(void* workspace, void* stream) {

@@ -218,6 +218,9 @@ __global__ void __launch_bounds__(384, 1)
           if (use > 0 && !mbar_wait(empty, (use - 1) & 1)) {
             record_status(a.status, kStatusTimeout); sh.abort_flag = 1; break;
           }
+          // Test hook (fp_debug_skip_k_load): the load is never issued, so the MMA issuer's
+          // bounded wait for it runs out and the kernel reports FP_ERR_TIMEOUT.
+          if (which == 0 && k == a.fault_skip_k && blockIdx.x == 0) continue;
           mbar_arrive_expect_tx(full, C::kKVBytes);
           uint8_t* dst = smem + (which == 0 ? C::kKOff : C::kVOff) + st * C::kKVBytes;
           const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;

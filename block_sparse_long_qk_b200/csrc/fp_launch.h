@@ -53,6 +53,7 @@ struct AttnArgs {
   int page_size, max_pages, num_pages;  // paged only
   int pair_heads;                       // 1: the two tiles of a CTA are two heads of one block
   int num_items;
+  int fault_skip_k;                     // test hook: CTA 0 skips the K load of this union block
   float scale_log2;                     // softmax scale * log2(e)
 };
 

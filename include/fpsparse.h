@@ -190,6 +190,16 @@ int fp_pool_and_mask_noalloc(const void* q, const void* k, int dtype, const floa
                              uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx,
                              void* stream);
 
+/*
+ * Test hook for the failure path (the pages have no counterpart). Makes the NEXT attention
+ * call issued from this thread skip, in its first CTA, the TMA load of K for the given union
+ * block (0 = the first block that CTA visits). That CTA's bounded pipeline wait then runs out
+ * after about 2 s and the call's workspace records FP_ERR_TIMEOUT (read it with
+ * fp_check_status); nothing faults and the context stays usable. One-shot: later calls are
+ * unaffected. Returns FP_ERR_INVALID_ARG for a negative index.
+ */
+int fp_debug_skip_k_load(int union_block);
+
 /* Bytes of device workspace the attention calls need (a fixed small size). */
 size_t fp_workspace_size(void);
 

@@ -228,6 +228,36 @@ def test_bad_index_is_reported_not_read(cuda_device):
     fp.check_status(cuda_device)   # cleared
 
 
+def test_pipeline_timeout_is_reported_and_cleared(cuda_device):
+    """A K load that never arrives (test hook, first CTA only): the MMA issuer's bounded wait
+    runs out, the status reads FP_ERR_TIMEOUT, the timeout is sticky until cleared, and the
+    next call on the same context is correct again."""
+    w = dataclasses.replace(W["llama32k"], Hq=2, Hkv=1, structure="iid")
+    inp = S.make_inputs(w, seed=5, seqlens=(256,))
+    keep = np.tril(np.ones((2, 2, 2), dtype=bool))
+    cnt, idx = keep_to_lists([keep], 2)
+    cnt, idx = cnt.to(cuda_device), idx.to(cuda_device)
+    q, k, v, _ = device_inputs(inp, cuda_device)
+    good, _ = fp.sparse_prefill_attn(q, k, v, cnt, idx, 128)
+    fp.check_status(cuda_device)
+    lib = fp.library()
+    assert lib.fp_debug_skip_k_load(-1) == -1
+    assert lib.fp_debug_skip_k_load(0) == 0
+    fp.sparse_prefill_attn(q, k, v, cnt, idx, 128)
+    # sticky: a launch on the same workspace before the check does no work at all
+    sentinel = torch.full_like(good, 7.0)
+    fp.sparse_prefill_attn(q, k, v, cnt, idx, 128, out=sentinel)
+    torch.cuda.synchronize()
+    assert bool((sentinel == 7.0).all())
+    with pytest.raises(fp.FpError) as e:
+        fp.check_status(cuda_device)
+    assert e.value.code == -4
+    # cleared by the check: the same call now completes and matches
+    again, _ = fp.sparse_prefill_attn(q, k, v, cnt, idx, 128)
+    fp.check_status(cuda_device)
+    assert torch.equal(again, good)
+
+
 def _full_size(name, cuda_device, n_rows=48):
     inp = S.make_inputs(name)
     w = inp.workload
