@@ -345,9 +345,10 @@ __global__ void __launch_bounds__(384, 1)
     // S row never has to stay in registers), packed and written over the S columns already
     // read; returns the row sum. Four independent partial sums keep the add chain short.
     // With e4m3 inputs the MMAs run twice as fast and the MUFU ex2 unit (4 lanes per clock per
-    // SM sub-partition) becomes the limit: there, one column pair in four off the diagonal takes
-    // the FMA-pipe polynomial instead (measured 7 % faster at 128K). With bf16 the extra FMA
-    // work costs more than it saves, so every exponential uses MUFU ex2.
+    // SM sub-partition) becomes the limit: there, three column pairs in eight off the diagonal
+    // take the FMA-pipe polynomial instead (measured at 128K: 8.10 ms vs 8.27 with 1/4, 8.57
+    // with 1/2, 8.76 with none). With bf16 the extra FMA work costs more than it saves, so
+    // every exponential uses MUFU ex2.
     constexpr bool kPolyExp = FP8;
     auto p_pass = [&](float mu, auto diag_tag) -> float {
       constexpr bool diag = decltype(diag_tag)::value;
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(384, 1)
               if (c0 + c > r) x.x = -INFINITY;
               if (c0 + c + 1 > r) x.y = -INFINITY;
             }
-            pp[c / 2] = (kPolyExp && !diag && (c / 2) % 4 == 3)
+            pp[c / 2] = (kPolyExp && !diag && (c / 2) % 8 >= 5)
                             ? exp2_poly2(x)
                             : make_float2(ex2(x.x), ex2(x.y));
           }
