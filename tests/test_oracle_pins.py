@@ -237,3 +237,74 @@ def test_per_head_scale_equals_prescaled_values():
     o2, _ = O.masked_causal_attention(q * qs[None, :, None], k * ks[None, :, None],
                                       v * vs[None, :, None], keep, cu, block, scale)
     assert np.array_equal(o1, o2)
+
+
+# ---- chunked (prefix-cached) prefill: the queries are the last q_len positions of each request
+
+def _chunked_case(seed=17):
+    kv_lens, q_lens = [70, 45, 33], [30, 45, 10]     # prefixes 40, 0, 23 (not block aligned)
+    ck = np.cumsum([0] + kv_lens).tolist()
+    cq = np.cumsum([0] + q_lens).tolist()
+    Hq, Hkv, d, block = 4, 2, 8, 16
+    qf = _rand((ck[-1], Hq, d), seed)                  # queries of every position
+    k, v = _rand((ck[-1], Hkv, d), seed + 1), _rand((ck[-1], Hkv, d), seed + 2)
+    rows = [r for b in range(3) for r in range(ck[b + 1] - q_lens[b], ck[b + 1])]
+    return qf, qf[rows], k, v, cq, ck, block
+
+
+def test_chunked_alpha0_equals_dense_rows_of_the_full_sequence():
+    """With every causal block kept, chunked attention of the last q_len queries equals the
+    matching rows of brute-force dense causal attention over the whole sequence."""
+    qf, q, k, v, cq, ck, block = _chunked_case()
+    scale = 1.0 / math.sqrt(q.shape[-1])
+    info, _ = O.query_blocks(cq, ck, block)
+    qp = O.pool_query_blocks(q, block, cq, ck)
+    kp = O.pool_blocks(k, block, ck)
+    sc = O.block_scores(qp, kp, cq, block, scale, cu_k=ck)
+    keeps = [O.block_keep(s, 0.0, row0=info[b][1]) for b, s in enumerate(sc)]
+    out, lse = O.masked_causal_attention(q, k, v, keeps, cq, block, scale, cu_k=ck)
+    bo, bl = _brute_attention(qf, k, v, ck, scale)
+    rows = [r for b in range(3) for r in range(ck[b + 1] - (cq[b + 1] - cq[b]), ck[b + 1])]
+    np.testing.assert_allclose(out, bo[rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, bl[:, rows], rtol=0, atol=1e-12)
+
+
+def test_chunked_query_pool_closed_form():
+    """x[t] = absolute position: a query block's mean is the mean of the positions it holds,
+    max(P0, I*B) .. min(L, (I+1)*B) - 1."""
+    kv_lens, q_lens, block = [70, 33], [30, 33], 16
+    ck = np.cumsum([0] + kv_lens).tolist()
+    cq = np.cumsum([0] + q_lens).tolist()
+    q = np.zeros((cq[-1], 1, 2))
+    for b in range(2):
+        P0 = kv_lens[b] - q_lens[b]
+        for i in range(q_lens[b]):
+            q[cq[b] + i] = P0 + i
+    p = O.pool_query_blocks(q, block, cq, ck)[0, :, 0]
+    expect = []
+    for b in range(2):
+        P0, L = kv_lens[b] - q_lens[b], kv_lens[b]
+        for I in range(P0 // block, (L + block - 1) // block):
+            lo, hi = max(P0, I * block), min(L, (I + 1) * block)
+            expect.append((lo + hi - 1) / 2.0)
+    np.testing.assert_array_equal(p, np.array(expect))
+
+
+def test_chunked_scores_and_keeps_match_the_full_prefill_on_whole_blocks():
+    """A query block that lies wholly inside the chunk pools the same queries as in a full
+    prefill, so its pooled row, its scores and its keep set are those of the full prefill."""
+    qf, q, k, v, cq, ck, block = _chunked_case(23)
+    scale = 1.0 / math.sqrt(q.shape[-1])
+    info, _ = O.query_blocks(cq, ck, block)
+    sc_c = O.block_scores(O.pool_query_blocks(q, block, cq, ck), O.pool_blocks(k, block, ck),
+                          cq, block, scale, cu_k=ck)
+    sc_f = O.block_scores(O.pool_blocks(qf, block, ck), O.pool_blocks(k, block, ck), ck,
+                          block, scale)
+    for b, (P0, I0, nq) in enumerate(info):
+        kc = O.block_keep(sc_c[b], 0.3, row0=I0)
+        kf = O.block_keep(sc_f[b], 0.3)
+        for i in range(nq):
+            I = I0 + i
+            if I * block >= P0:                       # whole block inside the chunk
+                assert np.array_equal(sc_c[b][:, i], sc_f[b][:, I])
+                assert np.array_equal(kc[:, i], kf[:, I])
