@@ -102,68 +102,100 @@ class Layer:
             self.paged = fp.PagedKV(inp.k_cache.to(dev), inp.v_cache.to(dev),
                                     inp.page_table.to(dev))
             self.k = self.v = None
-        self.batch = fp.Batch.make(w.seqlens, w.block, dev)
-        self.k_split = torch.empty(fp.k_split_shape(w.Hkv, self.batch.total_blocks, w.d),
-                                   dtype=torch.bfloat16, device=dev)
+        self.batch = self.cb = None
+        if w.q_lens is not None:
+            self.cb = fp.ChunkedBatch.make(w.q_lens, w.seqlens, w.block, dev)
+            nkb = self.cb.total_kblocks
+        else:
+            self.batch = fp.Batch.make(w.seqlens, w.block, dev)
+            nkb = self.batch.total_blocks
+        self.k_split = torch.empty(fp.k_split_shape(w.Hkv, nkb, w.d), dtype=torch.bfloat16,
+                                   device=dev)
         self.stream = torch.cuda.current_stream(dev)
         self.ev = []
 
     def step(self, events=None):
-        w, b = self.w, self.batch
+        w, b, cb = self.w, self.batch, self.cb
         sc = self.scales
         e = events
         if e is not None:
             e[0].record(self.stream)
-        qp, kp = fp.pool_qk(self.q, self.k, w.block, batch=b, q_scale=sc["q_scale"],
-                            k_scale=sc["k_scale"], paged=self.paged, k_split_out=self.k_split)
+        if cb is not None:
+            qp, kp = fp.pool_qk_chunked(self.q, self.k, cb, q_scale=sc["q_scale"],
+                                        k_scale=sc["k_scale"], paged=self.paged,
+                                        k_split_out=self.k_split)
+        else:
+            qp, kp = fp.pool_qk(self.q, self.k, w.block, batch=b, q_scale=sc["q_scale"],
+                                k_scale=sc["k_scale"], paged=self.paged,
+                                k_split_out=self.k_split)
         if e is not None:
             e[1].record(self.stream)
-        _, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b,
-                                          mask_bits=False, k_split=self.k_split)
+        if cb is not None:
+            _, cnt, idx = fp.build_block_mask_chunked(qp, kp, cb, w.alpha, mask_bits=False,
+                                                      k_split=self.k_split)
+        else:
+            _, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b,
+                                              mask_bits=False, k_split=self.k_split)
         if e is not None:
             e[2].record(self.stream)
-        if self.paged is not None:
-            out, _ = fp.sparse_prefill_attn_paged(self.q, self.paged, cnt, idx, b,
-                                                  q_scale=sc["q_scale"], k_scale=sc["k_scale"],
-                                                  v_scale=sc["v_scale"])
+        kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"])
+        if cb is not None:
+            out, _ = fp.sparse_prefill_attn_chunked(self.q, self.k, self.v, cnt, idx, cb,
+                                                    paged=self.paged, **kw)
+        elif self.paged is not None:
+            out, _ = fp.sparse_prefill_attn_paged(self.q, self.paged, cnt, idx, b, **kw)
         else:
             out, _ = fp.sparse_prefill_attn(self.q, self.k, self.v, cnt, idx, w.block, batch=b,
-                                            q_scale=sc["q_scale"], k_scale=sc["k_scale"],
-                                            v_scale=sc["v_scale"])
+                                            **kw)
         if e is not None:
             e[3].record(self.stream)
         return out, cnt, idx
 
 
-def work_counts(w, cnt, idx, batch):
+def _query_blocks(w):
+    """Per query block (all requests in order): absolute block I and the query positions
+    [lo, hi) it holds. Plain prefill is the case q_len = kv_len."""
+    B = w.block
+    q_lens = w.q_lens if w.q_lens is not None else w.seqlens
+    Is, los, his = [], [], []
+    for n, L in zip(q_lens, w.seqlens):
+        if n == 0:
+            continue
+        P0 = L - n
+        for I in range(P0 // B, (L + B - 1) // B):
+            Is.append(I)
+            los.append(max(P0, I * B))
+            his.append(min(L, (I + 1) * B))
+    return np.array(Is), np.array(los), np.array(his)
+
+
+def work_counts(w, cnt, idx, batch=None):
     """Algorithmic and executed attention FLOPs and the kept-block density of one layer."""
     B, d = w.block, w.d
-    cnt = cnt.long()
-    seq = torch.tensor(w.seqlens, device=cnt.device)
-    nb = (seq + B - 1) // B
-    # valid rows of each global block
-    nvalid = torch.cat([torch.clamp(L - torch.arange(n, device=cnt.device) * B, max=B)
-                        for L, n in zip(seq.tolist(), nb.tolist())])
-    blk_req = torch.repeat_interleave(torch.arange(len(w.seqlens), device=cnt.device), nb)
-    off = torch.cumsum(nb, 0) - nb
-    local = torch.arange(int(nb.sum()), device=cnt.device) - off[blk_req]
-    # kept blocks other than the diagonal are full B x n_I rectangles (earlier blocks of a
-    # request are full); the diagonal block contributes n(n+1)/2 causal pairs
-    pairs = (cnt - 1) * B * nvalid[None, :] + nvalid[None, :] * (nvalid[None, :] + 1) // 2
+    c = cnt.long().cpu().numpy()                       # [Hq, query blocks]
+    I, lo, hi = _query_blocks(w)
+    n = hi - lo
+    # a kept block below the diagonal is a full B-key block seen by the block's n queries;
+    # in the diagonal block the query at position p sees keys I*B .. p
+    a, b_ = lo - I * B, hi - I * B
+    diag = (b_ * (b_ + 1) - a * (a + 1)) // 2
+    pairs = (c - 1) * B * n[None, :] + diag[None, :]
     alg = 4.0 * d * float(pairs.sum())
-    executed = 4.0 * 128 * B * d * float(cnt.sum())
-    causal_blocks = float(((local + 1).sum()) * w.Hq)
-    return alg, executed, float(cnt.sum()) / causal_blocks
+    executed = 4.0 * 128 * B * d * float(c.sum())
+    causal_blocks = float((I + 1).sum()) * w.Hq
+    return alg, executed, float(c.sum()) / causal_blocks
 
 
 def pool_mask_bytes(w):
     eb = 1 if w.dtype == "e4m3" else 2
-    T = w.total_tokens
-    nblk = sum((L + w.block - 1) // w.block for L in w.seqlens)
+    Tk = w.total_tokens
+    Tq = sum(w.q_lens) if w.q_lens is not None else Tk
+    nkb = sum((L + w.block - 1) // w.block for L in w.seqlens)
+    nqb = len(_query_blocks(w)[0])
     # Q and K read once; pooled means written (fp32) and read back by the mask kernel, plus the
     # bf16 hi / lo split of the pooled keys written and read
-    return (T * (w.Hq + w.Hkv) * w.d * eb + 2 * nblk * (w.Hq + w.Hkv) * w.d * 4
-            + 2 * nblk * w.Hkv * w.d * 4)
+    return ((Tq * w.Hq + Tk * w.Hkv) * w.d * eb + 2 * (nqb * w.Hq + nkb * w.Hkv) * w.d * 4
+            + 2 * nkb * w.Hkv * w.d * 4)
 
 
 def cpu_baseline(inp, rows_sample=32, seed=5):
@@ -178,20 +210,25 @@ def cpu_baseline(inp, rows_sample=32, seed=5):
         cores = os.cpu_count()
     w = inp.workload
     cu = inp.cu_seqlens.tolist()
+    cu_q = inp.cu_q.tolist() if inp.cu_q is not None else cu
+    cu_k = cu if inp.cu_q is not None else None
     q, k, v = inp.codes_f32("q"), inp.codes_f32("k"), inp.codes_f32("v")
     qs, ks, vs = inp.scale_f64("q"), inp.scale_f64("k"), inp.scale_f64("v")
     scale = 1.0 / math.sqrt(w.d)
     t0 = time.perf_counter()
-    qp = O.pool_blocks(q, w.block, cu, scale=qs)
+    if cu_k is not None:
+        qp = O.pool_query_blocks(q, w.block, cu_q, cu_k, scale=qs)
+    else:
+        qp = O.pool_blocks(q, w.block, cu, scale=qs)
     kp = O.pool_blocks(k, w.block, cu, scale=ks)
-    sc = O.block_scores(qp, kp, cu, w.block, scale)
-    keeps = [O.block_keep(s, w.alpha) for s in sc]
+    sc = O.block_scores(qp, kp, cu_q, w.block, scale, cu_k=cu_k)
+    info, off = O.query_blocks(cu_q, cu_k, w.block)
+    keeps = [O.block_keep(s, w.alpha, row0=i[1]) for s, i in zip(sc, info)]
     t1 = time.perf_counter()
-    nb, off = O.request_blocks(cu, w.block)
     rng = np.random.default_rng(seed)
     rows = [(int(rng.integers(w.Hq)), int(rng.integers(off[-1]))) for _ in range(rows_sample)]
-    O.masked_causal_attention(q, k, v, keeps, cu, w.block, scale, rows=rows, q_scale=qs,
-                              k_scale=ks, v_scale=vs)
+    O.masked_causal_attention(q, k, v, keeps, cu_q, w.block, scale, rows=rows, q_scale=qs,
+                              k_scale=ks, v_scale=vs, cu_k=cu_k)
     t2 = time.perf_counter()
     total_rows = w.Hq * off[-1]
     ms = 1e3 * ((t1 - t0) + (t2 - t1) * total_rows / rows_sample)
@@ -253,7 +290,9 @@ def run_reference(args, world, rank):
 def _config(w, args):
     return {"workload": f"{w.name}: L={'+'.join(map(str, w.seqlens)) if len(w.seqlens) < 9 else w.total_tokens} "
                         f"Hq={w.Hq} Hkv={w.Hkv} d={w.d} block={w.block} alpha={w.alpha} "
-                        f"{w.dtype}" + (f" paged{w.page_size}" if w.page_size else ""),
+                        f"{w.dtype}" + (f" paged{w.page_size}" if w.page_size else "")
+                        + (f" chunked: q={sum(w.q_lens)} new tokens after cached prefixes"
+                           if w.q_lens is not None else ""),
             "tokens": w.total_tokens, "requests": w.batch, "parallelism": f"replicas{args.gpus}",
             "l2": "inputs larger than L2 (no flush)"}
 
@@ -293,7 +332,7 @@ def run_native(args, world, rank, local):
     attn_l = [e[2].elapsed_time(e[3]) for e in evs]
     pool_ms, mask_ms, attn_ms = (statistics.mean(x) for x in (pool_l, mask_l, attn_l))
 
-    alg, executed, density = work_counts(w, cnt, idx, layer.batch)
+    alg, executed, density = work_counts(w, cnt, idx)
     pm_bytes = pool_mask_bytes(w)
     peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     if w.dtype == "e4m3":

@@ -14,7 +14,9 @@ Ultra-Fast Long-Context Prefilling", technical summary section 2):
 
 ``sparse_prefill`` runs all three. Paged K/V (``PagedKV``) and varlen batches (``Batch``)
 follow "FlashPrefill V2: Block-Sparse Prefill Attention for Long-Context LLM Serving",
-Abstract (paged KV cache, continuous batching).
+Abstract (paged KV cache, continuous batching); so do the ``*_chunked`` calls with a
+``ChunkedBatch``, whose requests prefill only the last q_len of their kv_len positions (a
+chunk after a cached prefix).
 """
 from __future__ import annotations
 
@@ -29,7 +31,8 @@ import torch
 __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_attn",
            "sparse_prefill_attn_paged", "sparse_prefill", "check_status", "workspace",
            "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "header_symbols",
-           "pool_and_mask_noalloc", "k_split_shape"]
+           "pool_and_mask_noalloc", "k_split_shape", "ChunkedBatch", "pool_qk_chunked",
+           "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfpsparse.so")
@@ -59,6 +62,13 @@ _SIGNATURES = {
     "fp_debug_skip_k_load": (_i, [_i]),
     "fp_pool_and_mask_noalloc": (_i, [_p, _p, _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
                                       _i, _p, _i, _i, _i, _f, _f, _i, _p, _p, _p, _p]),
+    "fp_pool_qk_chunked": (_i, [_p, _p, _i, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
+                                _i, _i, _p, _i, _i, _i, _p, _p, _p, _p]),
+    "fp_build_block_mask_chunked": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
+                                         _i, _i, _f, _f, _i, _p, _p, _p, _p]),
+    "fp_sparse_prefill_attn_chunked": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _i, _i,
+                                            _i, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _i, _f,
+                                            _p, _p, _p, _p, _p, _p]),
 }
 
 
@@ -349,3 +359,142 @@ def pool_and_mask_noalloc(q, k, alpha=0.1, block=128, *, batch: Batch | None = N
         kk.shape[0] if pt is not None else 0, float(alpha), float(scale), int(flags),
         _ptr(bits), _ptr(kv_cnt), _ptr(kv_idx), _stream(dev)))
     return bits, kv_cnt, kv_idx
+
+
+@dataclasses.dataclass
+class ChunkedBatch:
+    """A chunked / prefix-cached varlen batch: request b has kv_lens[b] keys and prefills its
+    last q_lens[b] positions. Blocks lie on absolute positions; the query blocks of request b
+    are the absolute blocks (kv_len - q_len) // block .. ceil(kv_len / block) - 1."""
+    q_lens: tuple
+    kv_lens: tuple
+    block: int
+    cu_q: torch.Tensor        # int32 [B+1] on the device
+    cu_qblocks: torch.Tensor  # int32 [B+1]
+    cu_k: torch.Tensor        # int32 [B+1]
+    cu_kblocks: torch.Tensor  # int32 [B+1]
+    total_q: int
+    total_k: int
+    total_qblocks: int
+    total_kblocks: int
+    max_kblocks: int
+
+    @staticmethod
+    def make(q_lens, kv_lens, block, device):
+        q_lens = tuple(int(x) for x in q_lens)
+        kv_lens = tuple(int(x) for x in kv_lens)
+        if len(q_lens) != len(kv_lens) or not q_lens:
+            raise ValueError("q_lens and kv_lens need one entry per request")
+        nk, nq = [], []
+        for n, L in zip(q_lens, kv_lens):
+            if not 0 <= n <= L:
+                raise ValueError(f"q_len {n} must lie in [0, kv_len {L}]")
+            nk.append((L + block - 1) // block)
+            nq.append(nk[-1] - (L - n) // block if n > 0 else 0)
+
+        def cum(xs):
+            out = [0]
+            for x in xs:
+                out.append(out[-1] + x)
+            return out
+        cq, ck, cqb, ckb = cum(q_lens), cum(kv_lens), cum(nq), cum(nk)
+
+        def dev(xs):
+            return torch.tensor(xs, dtype=torch.int32, device=device)
+        return ChunkedBatch(q_lens, kv_lens, block, dev(cq), dev(cqb), dev(ck), dev(ckb),
+                            cq[-1], ck[-1], cqb[-1], ckb[-1], max(nk))
+
+    @property
+    def size(self):
+        return len(self.q_lens)
+
+    def _args(self):
+        return (_ptr(self.cu_q), _ptr(self.cu_qblocks), _ptr(self.cu_k), _ptr(self.cu_kblocks),
+                self.size)
+
+
+def pool_qk_chunked(q, k, cb: ChunkedBatch, *, q_scale=None, k_scale=None,
+                    paged: PagedKV | None = None, k_split_out=None):
+    """Block means for a chunked batch: q_pool [Hq, total_qblocks, d] over the queries each
+    query block holds, k_pool [Hkv, total_kblocks, d] over all keys (cached prefix included)."""
+    _, Hq, d = q.shape
+    kk = paged.k_cache if paged is not None else k
+    Hkv = kk.shape[-2]
+    q_pool = torch.empty((Hq, cb.total_qblocks, d), dtype=torch.float32, device=q.device)
+    k_pool = torch.empty((Hkv, cb.total_kblocks, d), dtype=torch.float32, device=q.device)
+    pt = paged.page_table if paged is not None else None
+    _check(library().fp_pool_qk_chunked(
+        _ptr(q), _ptr(kk), _dtype_code(q), _ptr(q_scale), _ptr(k_scale), *cb._args(),
+        cb.total_q, cb.total_k, cb.total_qblocks, cb.total_kblocks, Hq, Hkv, d, cb.block,
+        _ptr(pt), paged.page_size if paged else 0, pt.shape[1] if pt is not None else 0,
+        kk.shape[0] if pt is not None else 0, _ptr(q_pool), _ptr(k_pool), _ptr(k_split_out),
+        _stream(q.device)))
+    return q_pool, k_pool
+
+
+def build_block_mask_chunked(q_pool, k_pool, cb: ChunkedBatch, alpha=0.1, *, scale=None,
+                             flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True, k_split=None):
+    """Threshold for a chunked batch -> (mask_bits or None [Hq, total_qblocks, words],
+    kv_cnt [Hq, total_qblocks], kv_idx [Hq, total_qblocks, max_kblocks])."""
+    Hq, nqb, d = q_pool.shape
+    Hkv = k_pool.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dev = q_pool.device
+    words = (cb.max_kblocks + 31) // 32
+    bits = torch.zeros((Hq, nqb, words), dtype=torch.int32, device=dev) if mask_bits else None
+    kv_cnt = torch.empty((Hq, nqb), dtype=torch.int32, device=dev)
+    kv_idx = torch.empty((Hq, nqb, cb.max_kblocks), dtype=torch.int32, device=dev)
+    _check(library().fp_build_block_mask_chunked(
+        _ptr(q_pool), _ptr(k_pool), _ptr(k_split), *cb._args(), cb.total_qblocks,
+        cb.total_kblocks, cb.max_kblocks, Hq, Hkv, d, cb.block, float(alpha), float(scale),
+        int(flags), _ptr(bits), _ptr(kv_cnt), _ptr(kv_idx), _stream(dev)))
+    return bits, kv_cnt, kv_idx
+
+
+def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
+                                paged: PagedKV | None = None, scale=None, q_scale=None,
+                                k_scale=None, v_scale=None, return_lse=False, out=None, ws=None):
+    """Attention of the chunk's queries over the kept KV blocks of the whole request ->
+    (out bf16 [total_q, Hq, d], lse [Hq, total_q] or None). K/V are contiguous [total_k, Hkv,
+    d] (``k``, ``v``) or the caches of ``paged``."""
+    T, Hq, d = q.shape
+    kk = paged.k_cache if paged is not None else k
+    vv = paged.v_cache if paged is not None else v
+    Hkv = kk.shape[-2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if return_lse else None
+    ws = workspace(q.device) if ws is None else ws
+    pt = paged.page_table if paged is not None else None
+    _check(library().fp_sparse_prefill_attn_chunked(
+        _ptr(q), _ptr(kk), _ptr(vv), _dtype_code(q), _ptr(q_scale), _ptr(k_scale),
+        _ptr(v_scale), *cb._args(), cb.total_q, cb.total_k, cb.total_qblocks, cb.total_kblocks,
+        cb.max_kblocks, Hq, Hkv, d, cb.block, _ptr(pt), paged.page_size if paged else 0,
+        pt.shape[1] if pt is not None else 0, kk.shape[0] if pt is not None else 0,
+        float(scale), _ptr(kv_cnt), _ptr(kv_idx), _ptr(out), _ptr(lse), _ptr(ws),
+        _stream(q.device)))
+    return out, lse
+
+
+def sparse_prefill_chunked(q, k, v, cb: ChunkedBatch, alpha=0.1, *,
+                           paged: PagedKV | None = None, scale=None, q_scale=None,
+                           k_scale=None, v_scale=None, return_lse=False,
+                           flags=FORCE_FIRST | FORCE_DIAG):
+    """The whole path for a chunked batch. Returns (out, lse or None, kv_cnt, kv_idx)."""
+    d = q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    Hkv = (paged.k_cache if paged is not None else k).shape[-2]
+    k_split = torch.empty(k_split_shape(Hkv, cb.total_kblocks, d), dtype=torch.bfloat16,
+                          device=q.device)
+    q_pool, k_pool = pool_qk_chunked(q, k, cb, q_scale=q_scale, k_scale=k_scale, paged=paged,
+                                     k_split_out=k_split)
+    _, kv_cnt, kv_idx = build_block_mask_chunked(q_pool, k_pool, cb, alpha, scale=scale,
+                                                 flags=flags, mask_bits=False, k_split=k_split)
+    out, lse = sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb, paged=paged, scale=scale,
+                                           q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,
+                                           return_lse=return_lse)
+    return out, lse, kv_cnt, kv_idx

@@ -93,87 +93,108 @@ const char* fp_last_error_string(void) { return g_err.c_str(); }
 
 size_t fp_workspace_size(void) { return 256; }
 
-int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
-               const float* k_scale, const int32_t* cu_seqlens, const int32_t* cu_blocks,
-               int batch, int total_tokens, int total_blocks, int Hq, int Hkv, int d,
-               int block, const int32_t* k_page_table, int page_size, int max_pages,
-               int num_pages, float* q_pool, float* k_pool, void* k_pool_split, void* stream) {
-  g_err.clear();
-  int rc = check_common(dtype, q_scale, k_scale, nullptr, false, cu_seqlens, cu_blocks, batch,
-                        total_tokens, total_blocks, Hq, Hkv, d, block);
-  if (rc) return rc;
+}  // extern "C"
+
+namespace {
+
+// The varlen description of plain prefill: queries and keys are the same rows.
+fp::Seqs plain_seqs(const int32_t* cu_seqlens, const int32_t* cu_blocks, int batch,
+                    int total_tokens, int total_blocks, int max_blocks, int block) {
+  fp::Seqs s{};
+  s.cu_q = s.cu_k = cu_seqlens;
+  s.cu_qb = s.cu_kb = cu_blocks;
+  s.batch = batch;
+  s.total_q = s.total_k = total_tokens;
+  s.total_qb = s.total_kb = total_blocks;
+  s.max_kb = max_blocks;
+  s.block = block;
+  return s;
+}
+
+// Checks of a chunked varlen description (all four prefix-sum arrays are required).
+int check_chunked(const int32_t* cu_q, const int32_t* cu_qblocks, const int32_t* cu_k,
+                  const int32_t* cu_kblocks, int batch, int total_q, int total_k, int total_qb,
+                  int total_kb, int max_kb) {
+  if (batch < 1) return fail(FP_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", batch);
+  if (!cu_q || !cu_qblocks || !cu_k || !cu_kblocks)
+    return fail(FP_ERR_INVALID_ARG, "chunked prefill needs cu_q, cu_qblocks, cu_k, cu_kblocks");
+  if (total_q < 0 || total_k < 0 || total_qb < 0 || total_kb < 0 || max_kb < 0)
+    return fail(FP_ERR_INVALID_ARG, "negative token or block count");
+  if (total_q > total_k)
+    return fail(FP_ERR_INVALID_ARG, "total_q %d exceeds total_k %d", total_q, total_k);
+  if (total_qb > total_kb)
+    return fail(FP_ERR_INVALID_ARG, "total_qblocks %d exceeds total_kblocks %d", total_qb,
+                total_kb);
+  if (total_kb > 0 && max_kb < 1) return fail(FP_ERR_INVALID_ARG, "bad block counts");
+  return FP_OK;
+}
+
+int check_paging(const int32_t* page_table, int page_size, int max_pages, int num_pages,
+                 int block) {
+  if (page_table &&
+      (page_size < 16 || page_size % 16 || block % page_size || max_pages < 1 || num_pages < 1))
+    return fail(FP_ERR_INVALID_ARG, "page_size %d must be a multiple of 16 dividing block %d",
+                page_size, block);
+  return FP_OK;
+}
+
+int pool_impl(const void* q, const void* k, int dtype, const float* q_scale,
+              const float* k_scale, const fp::Seqs& s, int Hq, int Hkv, int d,
+              const int32_t* k_page_table, int page_size, int max_pages, int num_pages,
+              float* q_pool, float* k_pool, void* k_pool_split, void* stream) {
   if (!q || !k || !q_pool || !k_pool) return fail(FP_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool) ||
       !aligned16(k_pool_split))
     return fail(FP_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  if (k_page_table) {
-    if (page_size < 16 || page_size % 16 || block % page_size || max_pages < 1 || num_pages < 1)
-      return fail(FP_ERR_INVALID_ARG, "page_size %d must be a multiple of 16 dividing block %d",
-                  page_size, block);
-    if (cu_blocks == nullptr)
-      return fail(FP_ERR_INVALID_ARG, "a paged K needs cu_seqlens/cu_blocks");
-  }
-  if (total_blocks == 0) return FP_OK;
+  int rc = check_paging(k_page_table, page_size, max_pages, num_pages, s.block);
+  if (rc) return rc;
+  if (k_page_table && s.cu_k == nullptr)
+    return fail(FP_ERR_INVALID_ARG, "a paged K needs the varlen prefix sums");
+  if (s.total_kb == 0) return FP_OK;
   fp::PoolArgs a{};
-  a.num_pages = num_pages;
   a.q = static_cast<const uint8_t*>(q);
   a.k = static_cast<const uint8_t*>(k);
   a.q_scale = q_scale;
   a.k_scale = k_scale;
-  a.cu_seqlens = cu_seqlens;
-  a.cu_blocks = cu_blocks;
   a.page_table = k_page_table;
   a.q_pool = q_pool;
   a.k_pool = k_pool;
   a.k_split = static_cast<__nv_bfloat16*>(k_pool_split);
-  a.batch = batch;
-  a.total_tokens = total_tokens;
-  a.total_blocks = total_blocks;
+  a.s = s;
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.d = d;
-  a.block = block;
   a.page_size = page_size;
   a.max_pages = max_pages;
+  a.num_pages = num_pages;
   cudaError_t e = fp::launch_pool(a, dtype == FP_DTYPE_E4M3, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FP_OK : cuda_fail(e, "pool kernel launch");
 }
 
-int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_pool_split,
-                        const int32_t* cu_blocks, int batch, int total_blocks, int max_blocks,
-                        int Hq, int Hkv, int d, float alpha, float scale, int flags,
-                        uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* stream) {
-  g_err.clear();
+int mask_impl(const float* q_pool, const float* k_pool, const void* k_pool_split,
+              const fp::Seqs& s, int Hq, int Hkv, int d, float alpha, float scale, int flags,
+              uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* stream) {
   if (!q_pool || !k_pool || !kv_cnt || !kv_idx) return fail(FP_ERR_INVALID_ARG, "null pointer");
-  if (batch < 1 || (batch > 1 && !cu_blocks))
-    return fail(FP_ERR_INVALID_ARG, "batch > 1 needs cu_blocks");
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv)
     return fail(FP_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq, Hkv);
   if (d != 64 && d != 128) return fail(FP_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
   if (!(alpha >= 0.f && alpha <= 1.f)) return fail(FP_ERR_INVALID_ARG, "alpha must be in [0, 1]");
-  if (total_blocks < 0 || max_blocks < 0 || (total_blocks > 0 && max_blocks < 1))
-    return fail(FP_ERR_INVALID_ARG, "bad block counts");
-  if (cu_blocks == nullptr && max_blocks != total_blocks)
-    return fail(FP_ERR_INVALID_ARG, "one sequence: max_blocks must equal total_blocks");
   if (!aligned16(q_pool) || !aligned16(k_pool) || !aligned16(k_pool_split))
     return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
-  if (total_blocks == 0) return FP_OK;
+  if (s.total_qb == 0) return FP_OK;
   const int G = Hq / Hkv;
-  const int nb = fp::mask_blocks_per_cta(G, d, max_blocks);
+  const int nb = fp::mask_blocks_per_cta(G, d, s.max_kb);
   if (nb == 0 && !fp::mask_tc_supported(G, d))
     return fail(FP_ERR_UNSUPPORTED, "%d blocks per request with %d heads per KV head exceed the "
-                "shared-memory score rows of the mask kernel", max_blocks, G);
+                "shared-memory score rows of the mask kernel", s.max_kb, G);
   fp::MaskArgs a{};
   a.q_pool = q_pool;
   a.k_pool = k_pool;
   a.k_split = k_pool_split;
-  a.cu_blocks = cu_blocks;
   a.mask_bits = mask_bits;
   a.kv_cnt = kv_cnt;
   a.kv_idx = kv_idx;
-  a.batch = batch;
-  a.total_blocks = total_blocks;
-  a.max_blocks = max_blocks;
+  a.s = s;
   a.Hq = Hq;
   a.Hkv = Hkv;
   a.d = d;
@@ -186,39 +207,25 @@ int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_
   return e == cudaSuccess ? FP_OK : cuda_fail(e, "mask kernel launch");
 }
 
-static int attn_common(const void* q, const void* k, const void* v, int dtype,
-                       const float* q_scale, const float* k_scale, const float* v_scale,
-                       const int32_t* cu_seqlens, const int32_t* cu_blocks, int batch,
-                       int total_tokens, int total_blocks, int max_blocks, int Hq, int Hkv,
-                       int d, int block, const int32_t* page_table, int page_size,
-                       int max_pages, int num_pages, float scale, const int32_t* kv_cnt,
-                       const int32_t* kv_idx, void* out, float* lse, void* workspace,
-                       void* stream) {
-  g_err.clear();
-  int rc = check_common(dtype, q_scale, k_scale, v_scale, true, cu_seqlens, cu_blocks, batch,
-                        total_tokens, total_blocks, Hq, Hkv, d, block);
-  if (rc) return rc;
+int attn_impl(const void* q, const void* k, const void* v, int dtype, const float* q_scale,
+              const float* k_scale, const float* v_scale, const fp::Seqs& s, int Hq, int Hkv,
+              int d, const int32_t* page_table, int page_size, int max_pages, int num_pages,
+              float scale, const int32_t* kv_cnt, const int32_t* kv_idx, void* out, float* lse,
+              void* workspace, void* stream) {
   if (!q || !k || !v || !out || !kv_cnt || !kv_idx || !workspace)
     return fail(FP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(FP_ERR_INVALID_ARG, "Q, K, V and out must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(FP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  if (dtype == FP_DTYPE_E4M3 && !(d == 128 && block == 128))
+  if (dtype == FP_DTYPE_E4M3 && !(d == 128 && s.block == 128))
     return fail(FP_ERR_UNSUPPORTED, "e4m3 attention supports d = 128, block = 128");
-  if (cu_blocks == nullptr && max_blocks != total_blocks)
-    return fail(FP_ERR_INVALID_ARG, "one sequence: max_blocks must equal total_blocks");
-  if (page_table) {
-    if (page_size < 16 || page_size % 16 || block % page_size || max_pages < 1 || num_pages < 1)
-      return fail(FP_ERR_INVALID_ARG, "page_size %d must be a multiple of 16 dividing block %d",
-                  page_size, block);
-    if (cu_blocks == nullptr)
-      return fail(FP_ERR_INVALID_ARG, "paged attention needs cu_seqlens/cu_blocks");
-  }
+  int rc = check_paging(page_table, page_size, max_pages, num_pages, s.block);
+  if (rc) return rc;
+  if (page_table && s.cu_k == nullptr)
+    return fail(FP_ERR_INVALID_ARG, "paged attention needs the varlen prefix sums");
   const int G = Hq / Hkv;
   fp::AttnArgs a{};
-  a.cu_seqlens = cu_seqlens;
-  a.cu_blocks = cu_blocks;
   a.kv_cnt = kv_cnt;
   a.kv_idx = kv_idx;
   a.page_table = page_table;
@@ -228,18 +235,14 @@ static int attn_common(const void* q, const void* k, const void* v, int dtype,
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse = lse;
   a.status = static_cast<uint32_t*>(workspace);
-  a.batch = batch;
-  a.total_tokens = total_tokens;
-  a.total_blocks = total_blocks;
-  a.max_blocks = max_blocks;
+  a.s = s;
   a.Hq = Hq;
   a.Hkv = Hkv;
-  a.block = block;
   a.page_size = page_size;
   a.max_pages = max_pages;
   a.num_pages = num_pages;
   a.pair_heads = (G % 2 == 0) ? 1 : 0;
-  a.num_items = a.pair_heads ? (Hq / 2) * total_blocks : Hq * total_blocks;
+  a.num_items = a.pair_heads ? (Hq / 2) * s.total_qb : Hq * s.total_qb;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.fault_skip_k = g_fault_skip_k;
   g_fault_skip_k = -1;
@@ -250,12 +253,51 @@ static int attn_common(const void* q, const void* k, const void* v, int dtype,
   L.e4m3 = dtype == FP_DTYPE_E4M3;
   L.paged = page_table != nullptr;
   L.d = d;
-  L.kv_rows = page_table ? static_cast<long long>(num_pages) * page_size : total_tokens;
-  L.seg_rows = page_table ? page_size : block;
-  if (total_blocks == 0) return FP_OK;
-  cudaError_t e = fp::launch_attn(a, L, block, static_cast<cudaStream_t>(stream));
+  L.kv_rows = page_table ? static_cast<long long>(num_pages) * page_size : s.total_k;
+  L.seg_rows = page_table ? page_size : s.block;
+  if (s.total_qb == 0) return FP_OK;
+  cudaError_t e = fp::launch_attn(a, L, s.block, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return fail(FP_ERR_UNSUPPORTED, "unsupported d/block/dtype");
   return e == cudaSuccess ? FP_OK : cuda_fail(e, "attention kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
+               const float* k_scale, const int32_t* cu_seqlens, const int32_t* cu_blocks,
+               int batch, int total_tokens, int total_blocks, int Hq, int Hkv, int d,
+               int block, const int32_t* k_page_table, int page_size, int max_pages,
+               int num_pages, float* q_pool, float* k_pool, void* k_pool_split, void* stream) {
+  g_err.clear();
+  int rc = check_common(dtype, q_scale, k_scale, nullptr, false, cu_seqlens, cu_blocks, batch,
+                        total_tokens, total_blocks, Hq, Hkv, d, block);
+  if (rc) return rc;
+  return pool_impl(q, k, dtype, q_scale, k_scale,
+                   plain_seqs(cu_seqlens, cu_blocks, batch, total_tokens, total_blocks,
+                              total_blocks, block),
+                   Hq, Hkv, d, k_page_table, page_size, max_pages, num_pages, q_pool, k_pool,
+                   k_pool_split, stream);
+}
+
+int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_pool_split,
+                        const int32_t* cu_blocks, int batch, int total_blocks, int max_blocks,
+                        int Hq, int Hkv, int d, float alpha, float scale, int flags,
+                        uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* stream) {
+  g_err.clear();
+  if (batch < 1 || (batch > 1 && !cu_blocks))
+    return fail(FP_ERR_INVALID_ARG, "batch > 1 needs cu_blocks");
+  if (total_blocks < 0 || max_blocks < 0 || (total_blocks > 0 && max_blocks < 1))
+    return fail(FP_ERR_INVALID_ARG, "bad block counts");
+  if (cu_blocks == nullptr && max_blocks != total_blocks)
+    return fail(FP_ERR_INVALID_ARG, "one sequence: max_blocks must equal total_blocks");
+  // The mask needs only block indices: with no token counts, the query and key block lists of
+  // a plain prefill coincide (P0 = 0), which the block prefix sums alone describe.
+  const fp::Seqs s = plain_seqs(cu_blocks, cu_blocks, batch, total_blocks, total_blocks,
+                                max_blocks, 1);
+  return mask_impl(q_pool, k_pool, k_pool_split, s, Hq, Hkv, d, alpha, scale, flags, mask_bits,
+                   kv_cnt, kv_idx, stream);
 }
 
 int fp_sparse_prefill_attn(const void* q, const void* k, const void* v, int dtype,
@@ -265,9 +307,17 @@ int fp_sparse_prefill_attn(const void* q, const void* k, const void* v, int dtyp
                            int Hkv, int d, int block, float scale, const int32_t* kv_cnt,
                            const int32_t* kv_idx, void* out, float* lse, void* workspace,
                            void* stream) {
-  return attn_common(q, k, v, dtype, q_scale, k_scale, v_scale, cu_seqlens, cu_blocks, batch,
-                     total_tokens, total_blocks, max_blocks, Hq, Hkv, d, block, nullptr, 0, 0,
-                     0, scale, kv_cnt, kv_idx, out, lse, workspace, stream);
+  g_err.clear();
+  int rc = check_common(dtype, q_scale, k_scale, v_scale, true, cu_seqlens, cu_blocks, batch,
+                        total_tokens, total_blocks, Hq, Hkv, d, block);
+  if (rc) return rc;
+  if (cu_blocks == nullptr && max_blocks != total_blocks)
+    return fail(FP_ERR_INVALID_ARG, "one sequence: max_blocks must equal total_blocks");
+  return attn_impl(q, k, v, dtype, q_scale, k_scale, v_scale,
+                   plain_seqs(cu_seqlens, cu_blocks, batch, total_tokens, total_blocks,
+                              max_blocks, block),
+                   Hq, Hkv, d, nullptr, 0, 0, 0, scale, kv_cnt, kv_idx, out, lse, workspace,
+                   stream);
 }
 
 int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void* v_cache,
@@ -279,14 +329,103 @@ int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void*
                                  int max_pages, int num_pages, float scale,
                                  const int32_t* kv_cnt, const int32_t* kv_idx, void* out,
                                  float* lse, void* workspace, void* stream) {
-  if (!page_table) {
-    g_err = "paged attention needs a page table";
-    return FP_ERR_INVALID_ARG;
-  }
-  return attn_common(q, k_cache, v_cache, dtype, q_scale, k_scale, v_scale, cu_seqlens,
-                     cu_blocks, batch, total_tokens, total_blocks, max_blocks, Hq, Hkv, d,
-                     block, page_table, page_size, max_pages, num_pages, scale, kv_cnt, kv_idx,
-                     out, lse, workspace, stream);
+  g_err.clear();
+  if (!page_table) return fail(FP_ERR_INVALID_ARG, "paged attention needs a page table");
+  int rc = check_common(dtype, q_scale, k_scale, v_scale, true, cu_seqlens, cu_blocks, batch,
+                        total_tokens, total_blocks, Hq, Hkv, d, block);
+  if (rc) return rc;
+  if (cu_blocks == nullptr && max_blocks != total_blocks)
+    return fail(FP_ERR_INVALID_ARG, "one sequence: max_blocks must equal total_blocks");
+  return attn_impl(q, k_cache, v_cache, dtype, q_scale, k_scale, v_scale,
+                   plain_seqs(cu_seqlens, cu_blocks, batch, total_tokens, total_blocks,
+                              max_blocks, block),
+                   Hq, Hkv, d, page_table, page_size, max_pages, num_pages, scale, kv_cnt,
+                   kv_idx, out, lse, workspace, stream);
+}
+
+static fp::Seqs chunked_seqs(const int32_t* cu_q, const int32_t* cu_qblocks,
+                             const int32_t* cu_k, const int32_t* cu_kblocks, int batch,
+                             int total_q, int total_k, int total_qblocks, int total_kblocks,
+                             int max_kblocks, int block) {
+  fp::Seqs s{};
+  s.cu_q = cu_q;
+  s.cu_qb = cu_qblocks;
+  s.cu_k = cu_k;
+  s.cu_kb = cu_kblocks;
+  s.batch = batch;
+  s.total_q = total_q;
+  s.total_k = total_k;
+  s.total_qb = total_qblocks;
+  s.total_kb = total_kblocks;
+  s.max_kb = max_kblocks;
+  s.block = block;
+  return s;
+}
+
+int fp_pool_qk_chunked(const void* q, const void* k, int dtype, const float* q_scale,
+                       const float* k_scale, const int32_t* cu_q, const int32_t* cu_qblocks,
+                       const int32_t* cu_k, const int32_t* cu_kblocks, int batch, int total_q,
+                       int total_k, int total_qblocks, int total_kblocks, int Hq, int Hkv,
+                       int d, int block, const int32_t* k_page_table, int page_size,
+                       int max_pages, int num_pages, float* q_pool, float* k_pool,
+                       void* k_pool_split, void* stream) {
+  g_err.clear();
+  int rc = check_common(dtype, q_scale, k_scale, nullptr, false, cu_q, cu_qblocks, batch,
+                        total_q, total_qblocks, Hq, Hkv, d, block);
+  if (rc) return rc;
+  rc = check_chunked(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, total_q, total_k, total_qblocks,
+                     total_kblocks, total_kblocks > 0 ? 1 : 0);
+  if (rc) return rc;
+  return pool_impl(q, k, dtype, q_scale, k_scale,
+                   chunked_seqs(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, total_q, total_k,
+                                total_qblocks, total_kblocks, 0, block),
+                   Hq, Hkv, d, k_page_table, page_size, max_pages, num_pages, q_pool, k_pool,
+                   k_pool_split, stream);
+}
+
+int fp_build_block_mask_chunked(const float* q_pool, const float* k_pool,
+                                const void* k_pool_split, const int32_t* cu_q,
+                                const int32_t* cu_qblocks, const int32_t* cu_k,
+                                const int32_t* cu_kblocks, int batch, int total_qblocks,
+                                int total_kblocks, int max_kblocks, int Hq, int Hkv, int d,
+                                int block, float alpha, float scale, int flags,
+                                uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx,
+                                void* stream) {
+  g_err.clear();
+  if (block != 64 && block != 128)
+    return fail(FP_ERR_UNSUPPORTED, "block %d (supported: 64, 128)", block);
+  int rc = check_chunked(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, 0, 0, total_qblocks,
+                         total_kblocks, max_kblocks);
+  if (rc) return rc;
+  return mask_impl(q_pool, k_pool, k_pool_split,
+                   chunked_seqs(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, 0, 0, total_qblocks,
+                                total_kblocks, max_kblocks, block),
+                   Hq, Hkv, d, alpha, scale, flags, mask_bits, kv_cnt, kv_idx, stream);
+}
+
+int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, int dtype,
+                                   const float* q_scale, const float* k_scale,
+                                   const float* v_scale, const int32_t* cu_q,
+                                   const int32_t* cu_qblocks, const int32_t* cu_k,
+                                   const int32_t* cu_kblocks, int batch, int total_q,
+                                   int total_k, int total_qblocks, int total_kblocks,
+                                   int max_kblocks, int Hq, int Hkv, int d, int block,
+                                   const int32_t* page_table, int page_size, int max_pages,
+                                   int num_pages, float scale, const int32_t* kv_cnt,
+                                   const int32_t* kv_idx, void* out, float* lse,
+                                   void* workspace, void* stream) {
+  g_err.clear();
+  int rc = check_common(dtype, q_scale, k_scale, v_scale, true, cu_q, cu_qblocks, batch,
+                        total_q, total_qblocks, Hq, Hkv, d, block);
+  if (rc) return rc;
+  rc = check_chunked(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, total_q, total_k, total_qblocks,
+                     total_kblocks, max_kblocks);
+  if (rc) return rc;
+  return attn_impl(q, k, v, dtype, q_scale, k_scale, v_scale,
+                   chunked_seqs(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, total_q, total_k,
+                                total_qblocks, total_kblocks, max_kblocks, block),
+                   Hq, Hkv, d, page_table, page_size, max_pages, num_pages, scale, kv_cnt,
+                   kv_idx, out, lse, workspace, stream);
 }
 
 int fp_debug_skip_k_load(int union_block) {

@@ -56,7 +56,11 @@ struct AttnCfg {
 };
 
 struct Tile {
-  int h, Ig, I, q_lo, nvalid, cnt;  // nvalid = 0 marks an absent tile
+  // h: query head; Ig: global query block; I: its absolute block in the request (keys J <= I);
+  // q_lo: query row of tile row 0 (absolute position I * block; for the first block of a
+  // chunked request it precedes the request's first query row); rows r0 .. r1-1 are valid
+  // queries (r1 = 0 marks an absent tile); cnt / list: the kept-block list of (h, Ig).
+  int h, Ig, I, q_lo, r0, r1, cnt;
   const int32_t* list;
 };
 
@@ -101,44 +105,43 @@ struct UnionWalk {
   }
 };
 
-__device__ __forceinline__ void request_of(const AttnArgs& a, int Ig, int& b, int& base,
-                                           int& len, int& blk0) {
-  if (a.cu_blocks == nullptr) { b = 0; base = 0; len = a.total_tokens; blk0 = 0; return; }
-  b = find_request(a.cu_blocks, a.batch, Ig);
-  base = __ldg(a.cu_seqlens + b);
-  len = __ldg(a.cu_seqlens + b + 1) - base;
-  blk0 = __ldg(a.cu_blocks + b);
-}
-
-// Work item -> two tiles sharing one KV head. Items run heaviest-first (late query blocks
-// have the longest causal rows).
+// Work item -> two tiles sharing one KV head (and one request). Items run heaviest-first
+// (late query blocks have the longest causal rows). `kbase` / `len`: key row of the request's
+// position 0 and its key count; `b`: the request (page-table row).
 __device__ __forceinline__ void make_tiles(const AttnArgs& a, int item, Tile* t, int& g,
-                                           int& b, int& base, int& len) {
-  int blk0;
+                                           int& b, int& kbase, int& len) {
+  int Ig;
   if (a.pair_heads) {
     const int npairs = a.Hq / 2;
-    const int Ig = a.total_blocks - 1 - item / npairs;
+    Ig = a.s.total_qb - 1 - item / npairs;
     const int p = item % npairs;
-    request_of(a, Ig, b, base, len, blk0);
     for (int s = 0; s < 2; ++s) { t[s].h = 2 * p + s; t[s].Ig = Ig; }
   } else {
     // Query heads do not pair up on a KV head (odd group size): one tile per CTA.
-    const int Ig = a.total_blocks - 1 - item / a.Hq;
+    Ig = a.s.total_qb - 1 - item / a.Hq;
     const int h = item % a.Hq;
-    request_of(a, Ig, b, base, len, blk0);
     t[0].h = h; t[0].Ig = Ig;
     t[1].h = h; t[1].Ig = -1;
   }
+  const QBlock qb = query_block(a.s, Ig);
+  b = qb.b;
+  kbase = qb.kbase;
+  len = qb.L;
   g = t[0].h / (a.Hq / a.Hkv);
   for (int s = 0; s < 2; ++s) {
-    if (t[s].Ig < 0) { t[s].nvalid = 0; t[s].cnt = 0; t[s].list = a.kv_idx; t[s].I = -1; t[s].q_lo = 0; continue; }
-    t[s].I = t[s].Ig - blk0;
-    t[s].q_lo = base + t[s].I * a.block;
-    t[s].nvalid = min(a.block, len - t[s].I * a.block);
-    const size_t row = static_cast<size_t>(t[s].h) * a.total_blocks + t[s].Ig;
+    if (t[s].Ig < 0) {
+      t[s].r0 = t[s].r1 = 0; t[s].cnt = 0; t[s].list = a.kv_idx; t[s].I = -1; t[s].q_lo = 0;
+      continue;
+    }
+    const int B = a.s.block;
+    t[s].I = qb.I;
+    t[s].q_lo = qb.qrow0 + qb.I * B - qb.P0;
+    t[s].r0 = max(0, qb.P0 - qb.I * B);
+    t[s].r1 = min(B, qb.L - qb.I * B);
+    const size_t row = static_cast<size_t>(t[s].h) * a.s.total_qb + t[s].Ig;
     t[s].cnt = __ldg(a.kv_cnt + row);
-    t[s].cnt = max(0, min(t[s].cnt, a.max_blocks));
-    t[s].list = a.kv_idx + row * a.max_blocks;
+    t[s].cnt = max(0, min(t[s].cnt, a.s.max_kb));
+    t[s].list = a.kv_idx + row * a.s.max_kb;
   }
 }
 
@@ -162,8 +165,8 @@ __global__ void __launch_bounds__(384, 1)
   if (sh.abort_flag) return;
 
   Tile tl[2];
-  int g, b, base, len;
-  make_tiles(a, blockIdx.x, tl, g, b, base, len);
+  int g, b, kbase, len;
+  make_tiles(a, blockIdx.x, tl, g, b, kbase, len);
 
   if (threadIdx.x == 0) {
     mbar_init(&sh.q_full, 1);
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
-      const int ntiles = tl[1].nvalid > 0 ? 2 : 1;
+      const int ntiles = tl[1].r1 > 0 ? 2 : 1;
       mbar_arrive_expect_tx(&sh.q_full, ntiles * C::kQBytes);
       for (int s = 0; s < ntiles; ++s)
         for (int c = 0; c < C::kNChunk; ++c)
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(384, 1)
                 else record_status(a.status, kStatusBadIndex);
               }
             } else {
-              row = base + tok;
+              row = kbase + tok;
             }
             for (int c = 0; c < C::kNChunk; ++c)
               tma_load_3d(dst + c * (BN * 128) + sgi * (seg_rows * 128), tm, full,
@@ -337,10 +340,6 @@ __global__ void __launch_bounds__(384, 1)
     int n = 0;
     bool ok = true;
     int i = 0;
-    // P = 2^(s * sl2 - mu) for the whole row, packed and written over the S columns of TMEM;
-    // returns the row sum. Off the diagonal, one column pair in four takes the FMA-pipe
-    // polynomial instead of MUFU ex2, so the exponentials do not outrun the tensor core on
-    // the MUFU unit. Four independent partial sums keep the add chain short.
     // P = 2^(s * sl2 - mu) for the row, re-read from TMEM 64 columns at a time (so the whole
     // S row never has to stay in registers), packed and written over the S columns already
     // read; returns the row sum. Four independent partial sums keep the add chain short.
@@ -468,7 +467,7 @@ __global__ void __launch_bounds__(384, 1)
       if (n > 0) {
         float inv = (l > 0.f) ? 1.f / l : 0.f;
         if constexpr (FP8) inv *= __ldg(a.v_scale + g);
-        const bool valid = r < T.nvalid;
+        const bool valid = r >= T.r0 && r < T.r1;
         __nv_bfloat16* orow = a.out + (static_cast<size_t>(T.q_lo + r) * a.Hq + T.h) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -488,14 +487,14 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         if (valid && a.lse != nullptr)
-          a.lse[static_cast<size_t>(T.h) * a.total_tokens + T.q_lo + r] =
+          a.lse[static_cast<size_t>(T.h) * a.s.total_q + T.q_lo + r] =
               (l > 0.f) ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
-      } else if (r < T.nvalid) {
+      } else if (r >= T.r0 && r < T.r1) {
         // No kept block at all: the row attends to nothing; write zeros / -inf.
         __nv_bfloat16* orow = a.out + (static_cast<size_t>(T.q_lo + r) * a.Hq + T.h) * D;
         for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         if (a.lse != nullptr)
-          a.lse[static_cast<size_t>(T.h) * a.total_tokens + T.q_lo + r] = -INFINITY;
+          a.lse[static_cast<size_t>(T.h) * a.s.total_q + T.q_lo + r] = -INFINITY;
       }
     } else {
       record_status(a.status, kStatusTimeout);
@@ -536,7 +535,7 @@ template <int D, int BN, bool FP8, bool PAGED>
 static cudaError_t launch_t(const AttnArgs& a, const AttnLaunch& L, cudaStream_t stream) {
   using C = AttnCfg<D, BN, FP8>;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, L.q, FP8, D, a.Hq, a.total_tokens, 128) ||
+  if (!make_map(&mq, L.q, FP8, D, a.Hq, a.s.total_q, 128) ||
       !make_map(&mk, L.k, FP8, D, a.Hkv, L.kv_rows, L.seg_rows) ||
       !make_map(&mv, L.v, FP8, D, a.Hkv, L.kv_rows, L.seg_rows))
     return cudaErrorInvalidValue;

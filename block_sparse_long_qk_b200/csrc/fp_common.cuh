@@ -342,14 +342,4 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// Request of global block `gb` by binary search over cu_blocks (batch entries + 1).
-__device__ __forceinline__ int find_request(const int32_t* cu_blocks, int batch, int gb) {
-  int lo = 0, hi = batch - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (__ldg(cu_blocks + mid) <= gb) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
 }  // namespace fp

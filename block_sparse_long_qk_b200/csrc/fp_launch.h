@@ -8,38 +8,50 @@
 
 namespace fp {
 
+// A varlen batch whose queries may be a suffix of each request (chunked / prefix-cached
+// prefill): request b holds kv_len_b = cu_k[b+1] - cu_k[b] keys and q_len_b query rows, the
+// queries being the last q_len_b positions P0_b = kv_len_b - q_len_b .. kv_len_b - 1. Blocks
+// are defined on absolute positions: the request's KV blocks are 0 .. ceil(kv_len/block) - 1,
+// its query blocks run from I0_b = P0_b / block to the same last block. With cu_q == nullptr
+// the batch is one sequence of total_q = total_k tokens (P0 = 0). The entry points for plain
+// prefill pass the same arrays for queries and keys (P0 = 0 everywhere).
+struct Seqs {
+  const int32_t* cu_q;   // [batch + 1] query rows
+  const int32_t* cu_qb;  // [batch + 1] query blocks
+  const int32_t* cu_k;   // [batch + 1] key rows
+  const int32_t* cu_kb;  // [batch + 1] key blocks
+  int batch, total_q, total_k, total_qb, total_kb, max_kb, block;
+};
+
 struct PoolArgs {
   const uint8_t* q;
   const uint8_t* k;
   const float* q_scale;
   const float* k_scale;
-  const int32_t* cu_seqlens;
-  const int32_t* cu_blocks;
   const int32_t* page_table;
-  float* q_pool;
-  float* k_pool;
-  __nv_bfloat16* k_split;  // optional bf16 [2][Hkv][total_blocks][d] hi / lo parts of k_pool
-  int batch, total_tokens, total_blocks, Hq, Hkv, d, block, page_size, max_pages, num_pages;
+  float* q_pool;           // [Hq][total_qb][d]
+  float* k_pool;           // [Hkv][total_kb][d]
+  __nv_bfloat16* k_split;  // optional bf16 [2][Hkv][total_kb][d] hi / lo parts of k_pool
+  Seqs s;
+  int Hq, Hkv, d, page_size, max_pages, num_pages;
   int q_slices;  // column slices of Q per block (the rest of gridDim.y are K slices)
 };
 
 struct MaskArgs {
   const float* q_pool;
   const float* k_pool;
-  const void* k_split;  // bf16 [2][Hkv][total_blocks][d] hi / lo parts of k_pool, or nullptr
-  const int32_t* cu_blocks;
-  uint32_t* mask_bits;
-  int32_t* kv_cnt;
-  int32_t* kv_idx;
-  int batch, total_blocks, max_blocks, Hq, Hkv, d, G, NB;
+  const void* k_split;  // bf16 [2][Hkv][total_kb][d] hi / lo parts of k_pool, or nullptr
+  uint32_t* mask_bits;  // [Hq][total_qb][ceil(max_kb / 32)]
+  int32_t* kv_cnt;      // [Hq][total_qb]
+  int32_t* kv_idx;      // [Hq][total_qb][max_kb]
+  Seqs s;
+  int Hq, Hkv, d, G, NB;
   float log_alpha;  // -inf for alpha = 0
   float scale;
   int flags;
 };
 
 struct AttnArgs {
-  const int32_t* cu_seqlens;
-  const int32_t* cu_blocks;
   const int32_t* kv_cnt;
   const int32_t* kv_idx;
   const int32_t* page_table;
@@ -49,7 +61,8 @@ struct AttnArgs {
   __nv_bfloat16* out;
   float* lse;
   uint32_t* status;
-  int batch, total_tokens, total_blocks, max_blocks, Hq, Hkv, block;
+  Seqs s;
+  int Hq, Hkv;
   int page_size, max_pages, num_pages;  // paged only
   int pair_heads;                       // 1: the two tiles of a CTA are two heads of one block
   int num_items;
@@ -61,13 +74,13 @@ struct AttnLaunch {
   const void *q, *k, *v;
   bool e4m3, paged;
   int d;
-  long long kv_rows;  // rows of the K/V tensor map (T, or num_pages * page_size)
+  long long kv_rows;  // rows of the K/V tensor map (total_k, or num_pages * page_size)
   int seg_rows;       // rows per K/V TMA box (block, or page_size)
 };
 
 cudaError_t launch_pool(const PoolArgs& a, bool e4m3, cudaStream_t stream);
 cudaError_t launch_mask(const MaskArgs& a, cudaStream_t stream);
-int mask_blocks_per_cta(int G, int d, int max_blocks);
+int mask_blocks_per_cta(int G, int d, int max_kb);
 bool mask_tc_supported(int G, int d);   // tensor-core scores (mask_tc.cu) apply
 cudaError_t launch_mask_tc(const MaskArgs& a, cudaStream_t stream);
 cudaError_t launch_attn(const AttnArgs& a, const AttnLaunch& L, int block, cudaStream_t stream);
@@ -82,5 +95,62 @@ EncodeTiledFn tensor_map_encoder();
 
 // Records a printf-style message for fp_last_error_string() on this thread; returns `code`.
 int set_error(int code, const char* fmt, ...);
+
+}  // namespace fp
+
+namespace fp {
+
+// Query block gq of a batch: request b, absolute block index I, the request's first query
+// position P0 and key count L, the query row holding absolute position P0 (qrow0), the key row
+// of position 0 (kbase) and the global KV block of the request's block 0 (kb0).
+struct QBlock {
+  int b, I, P0, L, qrow0, kbase, kb0;
+};
+
+#ifdef __CUDACC__
+__device__ __forceinline__ int seqs_find(const int32_t* cu, int batch, int x) {
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ QBlock query_block(const Seqs& s, int gq) {
+  QBlock r;
+  if (s.cu_q == nullptr) {
+    r.b = 0; r.P0 = 0; r.L = s.total_k; r.qrow0 = 0; r.kbase = 0; r.kb0 = 0; r.I = gq;
+    return r;
+  }
+  r.b = seqs_find(s.cu_qb, s.batch, gq);
+  r.qrow0 = __ldg(s.cu_q + r.b);
+  const int nq = __ldg(s.cu_q + r.b + 1) - r.qrow0;
+  r.kbase = __ldg(s.cu_k + r.b);
+  r.L = __ldg(s.cu_k + r.b + 1) - r.kbase;
+  r.P0 = r.L - nq;
+  r.kb0 = __ldg(s.cu_kb + r.b);
+  r.I = r.P0 / s.block + (gq - __ldg(s.cu_qb + r.b));
+  return r;
+}
+
+// KV block gk of a batch: request b, block index J, key count L, key row of position 0.
+struct KBlock {
+  int b, J, L, kbase;
+};
+
+__device__ __forceinline__ KBlock key_block(const Seqs& s, int gk) {
+  KBlock r;
+  if (s.cu_k == nullptr) {
+    r.b = 0; r.J = gk; r.L = s.total_k; r.kbase = 0;
+    return r;
+  }
+  r.b = seqs_find(s.cu_kb, s.batch, gk);
+  r.kbase = __ldg(s.cu_k + r.b);
+  r.L = __ldg(s.cu_k + r.b + 1) - r.kbase;
+  r.J = gk - __ldg(s.cu_kb + r.b);
+  return r;
+}
+#endif
 
 }  // namespace fp

@@ -39,8 +39,8 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
   const int dp = mask_pad(a.d);
   float* sq = sm;                                  // [R][dp]
   float* sk = sq + static_cast<size_t>(R) * dp;    // [kMaskChunk][dp]
-  float* ss = sk + static_cast<size_t>(kMaskChunk) * dp;  // [R][max_blocks]
-  int* row_I = reinterpret_cast<int*>(ss + static_cast<size_t>(R) * a.max_blocks);
+  float* ss = sk + static_cast<size_t>(kMaskChunk) * dp;  // [R][max_kb]
+  int* row_I = reinterpret_cast<int*>(ss + static_cast<size_t>(R) * a.s.max_kb);
   int* row_kb = row_I + R;    // global block index of the row's request block 0
   int* row_h = row_kb + R;
   int* row_g = row_h + R;     // global query block (-1 if past the end)
@@ -53,11 +53,10 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
   for (int r = tid; r < R; r += kMaskThreads) {
     const int Ig = Ig0 + r / a.G;
     const int h = g * a.G + r % a.G;
-    if (Ig < a.total_blocks) {
-      int kb = 0;
-      if (a.cu_blocks != nullptr) kb = __ldg(a.cu_blocks + find_request(a.cu_blocks, a.batch, Ig));
-      row_I[r] = Ig - kb;
-      row_kb[r] = kb;
+    if (Ig < a.s.total_qb) {
+      const QBlock qb = query_block(a.s, Ig);
+      row_I[r] = qb.I;     // absolute query block: keys J = 0 .. I of the request
+      row_kb[r] = qb.kb0;  // global KV block of the request's block 0
       row_g[r] = Ig;
     } else {
       row_I[r] = -1;
@@ -72,17 +71,18 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
     const int r = i / d4, c = (i % d4) * 4;
     const int Ig = Ig0 + r / a.G;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (Ig < a.total_blocks)
+    if (Ig < a.s.total_qb)
       v = __ldg(reinterpret_cast<const float4*>(
-          a.q_pool + (static_cast<size_t>(g * a.G + r % a.G) * a.total_blocks + Ig) * a.d + c));
+          a.q_pool + (static_cast<size_t>(g * a.G + r % a.G) * a.s.total_qb + Ig) * a.d + c));
     *reinterpret_cast<float4*>(sq + r * dp + c) = v;
   }
   __syncthreads();
 
-  // Key-block range this CTA needs: from block 0 of its first row's request to its last row.
-  const int last_row_blk = min(Ig0 + a.NB, a.total_blocks) - 1;
+  // Key-block range this CTA needs: from block 0 of its first row's request to the diagonal
+  // block of its last row.
+  const int r_last = (min(Ig0 + a.NB, a.s.total_qb) - 1 - Ig0) * a.G;
   const int Jg_lo = row_kb[0];
-  const int Jg_hi = last_row_blk;
+  const int Jg_hi = row_kb[r_last] + row_I[r_last];
 
   // Thread -> (key column within the chunk, row group); rows rg, rg + 4, ... of the R rows.
   const int col = tid % kMaskChunk;
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j < nchunk)
         v = __ldg(reinterpret_cast<const float4*>(
-            a.k_pool + (static_cast<size_t>(g) * a.total_blocks + Jg0 + j) * a.d + c));
+            a.k_pool + (static_cast<size_t>(g) * a.s.total_kb + Jg0 + j) * a.d + c));
       *reinterpret_cast<float4*>(sk + j * dp + c) = v;
     }
     __syncthreads();
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
           const int r = r0 + u * kRowGroups;
           if (r < R && row_g[r] >= 0) {
             const int J = Jg - row_kb[r];
-            if (J >= 0 && J <= row_I[r]) ss[static_cast<size_t>(r) * a.max_blocks + J] = acc[u] * a.scale;
+            if (J >= 0 && J <= row_I[r]) ss[static_cast<size_t>(r) * a.s.max_kb + J] = acc[u] * a.scale;
           }
         }
       }
@@ -137,19 +137,19 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
 
   // Threshold, bits and compaction: one warp per row.
   const int warp = tid / 32, lane = tid % 32;
-  const int words = (a.max_blocks + 31) / 32;
+  const int words = (a.s.max_kb + 31) / 32;
   for (int r = warp; r < R; r += kMaskThreads / 32) {
     const int Ig = row_g[r];
     if (Ig < 0) continue;
     const int I = row_I[r];
     const int h = row_h[r];
-    const float* srow = ss + static_cast<size_t>(r) * a.max_blocks;
+    const float* srow = ss + static_cast<size_t>(r) * a.s.max_kb;
     float m = -INFINITY;
     for (int J = lane; J <= I; J += 32) m = fmaxf(m, srow[J]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const size_t row = static_cast<size_t>(h) * a.total_blocks + Ig;
-    int32_t* idx = a.kv_idx + row * a.max_blocks;
+    const size_t row = static_cast<size_t>(h) * a.s.total_qb + Ig;
+    int32_t* idx = a.kv_idx + row * a.s.max_kb;
     int cnt = 0;
     for (int w = 0; w < words; ++w) {
       const int J = w * 32 + lane;
@@ -179,11 +179,11 @@ int mask_blocks_per_cta(int G, int d, int max_blocks) {
 cudaError_t launch_mask(const MaskArgs& in, cudaStream_t stream) {
   if (mask_tc_supported(in.G, in.d)) return launch_mask_tc(in, stream);
   MaskArgs a = in;
-  const size_t smem = mask_smem_bytes(a.G * a.NB, a.d, a.max_blocks);
+  const size_t smem = mask_smem_bytes(a.G * a.NB, a.d, a.s.max_kb);
   cudaError_t e = cudaFuncSetAttribute(mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.total_blocks + a.NB - 1) / a.NB, a.Hkv);
+  dim3 grid((a.s.total_qb + a.NB - 1) / a.NB, a.Hkv);
   mask_kernel<<<grid, kMaskThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }

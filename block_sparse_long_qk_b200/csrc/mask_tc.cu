@@ -71,7 +71,7 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 
 // kTma: the B operand (pooled keys, split into bf16 hi / lo) is read by TMA from the split that
-// the pool kernel wrote (`tm_split`: 2-D map over [2 * Hkv * total_blocks, d] bf16 with
+// the pool kernel wrote (`tm_split`: 2-D map over [2 * Hkv * total_kb, d] bf16 with
 // 128-row, 64-column boxes), instead of being converted from fp32 by the threads.
 template <int D, bool kTma>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -100,10 +100,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid < kTcRows) {
     const int Ig = Ig0 + tid / a.G;
     row_h[tid] = g * a.G + tid % a.G;
-    if (Ig < a.total_blocks) {
-      const int kb = a.cu_blocks ? __ldg(a.cu_blocks + find_request(a.cu_blocks, a.batch, Ig)) : 0;
-      row_I[tid] = Ig - kb;
-      row_kb[tid] = kb;
+    if (Ig < a.s.total_qb) {
+      const QBlock qb = query_block(a.s, Ig);
+      row_I[tid] = qb.I;     // absolute query block: keys J = 0 .. I of the request
+      row_kb[tid] = qb.kb0;  // global KV block of the request's block 0
       row_g[tid] = Ig;
     } else {
       row_I[tid] = -1;
@@ -121,12 +121,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   // The CTA owns its 128 rows of mask words: zero them, keep bits are OR-ed in later.
   if (a.mask_bits != nullptr) {
-    const int words = (a.max_blocks + 31) / 32;
+    const int words = (a.s.max_kb + 31) / 32;
     for (int i = tid; i < kTcRows * words; i += kTcThreads) {
       const int rr = i / words;
       const int Ig = Ig0 + rr / a.G;
-      if (Ig < a.total_blocks)
-        a.mask_bits[(static_cast<size_t>(g * a.G + rr % a.G) * a.total_blocks + Ig) * words +
+      if (Ig < a.s.total_qb)
+        a.mask_bits[(static_cast<size_t>(g * a.G + rr % a.G) * a.s.total_qb + Ig) * words +
                     i % words] = 0u;
     }
   }
@@ -141,9 +141,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int r = u / kUnits, k0 = (u % kUnits) * 8;
     const int Ig = Ig0 + r / a.G;
     float v[8];
-    if (Ig < a.total_blocks) {
+    if (Ig < a.s.total_qb) {
       const float4* src = reinterpret_cast<const float4*>(
-          a.q_pool + (static_cast<size_t>(g * a.G + r % a.G) * a.total_blocks + Ig) * D + k0);
+          a.q_pool + (static_cast<size_t>(g * a.G + r % a.G) * a.s.total_qb + Ig) * D + k0);
       const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
       v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
       v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
@@ -158,8 +158,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Key-block range of the CTA: block 0 of its first row's request .. its last row's block.
-  const int last = min(Ig0 + rows_blk, a.total_blocks) - 1;
+  // Key-block range of the CTA: block 0 of its first row's request .. the diagonal block of
+  // its last row (rows are ordered by request, then by block).
+  const int r_last = (min(Ig0 + rows_blk, a.s.total_qb) - 1 - Ig0) * a.G;
+  const int last = row_kb[r_last] + row_I[r_last];
   const int Jg_lo = row_kb[0];
   const int nch = (last - Jg_lo) / kTcKeys + 1;
   const int W = 2 * nch;  // pass 0 chunks, then pass 1 chunks
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int Jg = Jg0 + j;
       if (Jg <= last) {
         const float4* src = reinterpret_cast<const float4*>(
-            a.k_pool + (static_cast<size_t>(g) * a.total_blocks + Jg) * D + k0);
+            a.k_pool + (static_cast<size_t>(g) * a.s.total_kb + Jg) * D + k0);
         xk[p][0] = __ldg(src);
         xk[p][1] = __ldg(src + 1);
       } else {
@@ -198,12 +200,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   };
 
-  // One chunk of the B operand by TMA: hi rows g * total_blocks + Jg0 .. +127 and the same rows
+  // One chunk of the B operand by TMA: hi rows g * total_kb + Jg0 .. +127 and the same rows
   // of the lo plane (rows past the group's last block carry other data or zeros; their score
   // columns are never valid).
   auto tma_chunk = [&](int w, int buf) {
-    const int row = g * a.total_blocks + Jg_lo + (w % nch) * kTcKeys;
-    const int lo_row = a.Hkv * a.total_blocks + row;
+    const int row = g * a.s.total_kb + Jg_lo + (w % nch) * kTcKeys;
+    const int lo_row = a.Hkv * a.s.total_kb + row;
     uint8_t* bh = smem + C::kB + (2 * buf) * C::kTile;
     uint8_t* bl = bh + C::kTile;
     mbar_arrive_expect_tx(&full[buf], C::kSplitTx);
@@ -243,9 +245,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int cnt = 0;                     // kept blocks of the row so far (same in all 4 threads)
   uint32_t pend_km = 0;            // keep bits of the previous chunk, written one chunk later
   int pend_J = 0, pend_item = -1;
-  const int words = (a.max_blocks + 31) / 32;
-  const size_t row = I >= 0 ? static_cast<size_t>(row_h[r]) * a.total_blocks + row_g[r] : 0;
-  int32_t* idx = a.kv_idx + row * a.max_blocks;
+  const int words = (a.s.max_kb + 31) / 32;
+  const size_t row = I >= 0 ? static_cast<size_t>(row_h[r]) * a.s.total_qb + row_g[r] : 0;
+  int32_t* idx = a.kv_idx + row * a.s.max_kb;
   uint32_t* bits_row = a.mask_bits ? a.mask_bits + row * words : nullptr;
 
   // Writes the previous chunk's kept indices at their place in the ascending list, using the
@@ -403,14 +405,14 @@ static cudaError_t launch_tc(const MaskArgs& a, const CUtensorMap& map, dim3 gri
 
 cudaError_t launch_mask_tc(const MaskArgs& a, cudaStream_t stream) {
   const int rows_blk = kTcRows / a.G;
-  dim3 grid(((a.total_blocks + rows_blk - 1) / rows_blk) * a.Hkv);
+  dim3 grid(((a.s.total_qb + rows_blk - 1) / rows_blk) * a.Hkv);
   CUtensorMap map;
   memset(&map, 0, sizeof(map));
   if (a.k_split != nullptr) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (enc == nullptr) return cudaErrorNotSupported;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.d),
-                          2ull * static_cast<cuuint64_t>(a.Hkv) * a.total_blocks};
+                          2ull * static_cast<cuuint64_t>(a.Hkv) * a.s.total_kb};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.d) * 2};
     cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(kTcKeys)};
     cuuint32_t estr[2] = {1u, 1u};

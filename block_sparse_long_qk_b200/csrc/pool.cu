@@ -5,6 +5,8 @@
 // the query skeleton is read as block means of Q as well, so that the pooled score of stage 2
 // equals the mean of the raw scaled Q K^T block (the fused 2-D reduction).
 //
+// Chunked prefill: query blocks hold only the request's query positions (see Seqs).
+//
 // HBM-bound stream: every CTA owns one (global block, tensor, 2 KB-wide column slice) and
 // its 128 threads each own 16 contiguous bytes of the token row (8 bf16 or 16 e4m3 values),
 // walking the block's tokens with 8 independent 16-byte loads in flight per thread. A warp
@@ -27,16 +29,25 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
   const int col = (slice * kPoolThreads + threadIdx.x) * EPT;
   if (col >= cols) return;
 
-  int b = 0, base = 0, len = a.total_tokens, blk0 = 0;
-  if (a.cu_blocks != nullptr) {
-    b = find_request(a.cu_blocks, a.batch, gb);
-    base = __ldg(a.cu_seqlens + b);
-    len = __ldg(a.cu_seqlens + b + 1) - base;
-    blk0 = __ldg(a.cu_blocks + b);
+  // Query block gb: the query positions it holds (chunked prefill: only those at or after
+  // the request's first query position P0). Key block gb: its keys, in a paged cache or at
+  // contiguous rows.
+  if (gb >= (is_q ? a.s.total_qb : a.s.total_kb)) return;
+  int n, b = 0, t0 = 0;
+  size_t first_row = 0;
+  if (is_q) {
+    const QBlock qb = query_block(a.s, gb);
+    const int lo = max(qb.P0, qb.I * a.s.block);
+    const int hi = min(qb.L, (qb.I + 1) * a.s.block);
+    n = hi - lo;
+    first_row = static_cast<size_t>(qb.qrow0) + (lo - qb.P0);
+  } else {
+    const KBlock kb = key_block(a.s, gb);
+    b = kb.b;
+    t0 = kb.J * a.s.block;
+    n = min(a.s.block, kb.L - t0);
+    first_row = static_cast<size_t>(kb.kbase) + t0;
   }
-  const int I = gb - blk0;
-  const int t0 = I * a.block;                      // request-local first token
-  const int n = min(a.block, len - t0);            // valid tokens of this block
   const uint8_t* src = is_q ? a.q : a.k;
   const bool paged = (!is_q) && a.page_table != nullptr;
   const size_t row_bytes = static_cast<size_t>(cols) * (E4M3 ? 1 : 2);
@@ -59,7 +70,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
       if (page < 0 || page >= a.num_pages) return nullptr;
       row = static_cast<size_t>(page) * a.page_size + (tl % a.page_size);
     } else {
-      row = static_cast<size_t>(base) + t0 + r0;
+      row = first_row + r0;
     }
     return src + row * row_bytes + col_bytes;
   };
@@ -109,7 +120,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
   const float* scale = is_q ? a.q_scale : a.k_scale;
   if (scale != nullptr) s *= __ldg(scale + h);
   float* dst = (is_q ? a.q_pool : a.k_pool) +
-               (static_cast<size_t>(h) * a.total_blocks + gb) * a.d + c;
+               (static_cast<size_t>(h) * (is_q ? a.s.total_qb : a.s.total_kb) + gb) * a.d + c;
 #pragma unroll
   for (int i = 0; i < EPT; ++i) acc[i] *= s;
 #pragma unroll
@@ -117,8 +128,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
     *reinterpret_cast<float4*>(dst + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
   if (!is_q && a.k_split != nullptr) {
     // bf16 hi / lo split of the pooled key (the tensor-core operands of the mask kernel).
-    const size_t plane = static_cast<size_t>(a.Hkv) * a.total_blocks * a.d;
-    __nv_bfloat16* hi = a.k_split + (static_cast<size_t>(h) * a.total_blocks + gb) * a.d + c;
+    const size_t plane = static_cast<size_t>(a.Hkv) * a.s.total_kb * a.d;
+    __nv_bfloat16* hi = a.k_split + (static_cast<size_t>(h) * a.s.total_kb + gb) * a.d + c;
 #pragma unroll
     for (int i = 0; i < EPT; i += 8) {
       uint32_t hw[4], lw[4];
@@ -141,7 +152,7 @@ cudaError_t launch_pool(const PoolArgs& in, bool e4m3, cudaStream_t stream) {
   const int per_cta = kPoolThreads * ept;
   a.q_slices = (a.Hq * a.d + per_cta - 1) / per_cta;
   const int k_slices = (a.Hkv * a.d + per_cta - 1) / per_cta;
-  dim3 grid(a.total_blocks, a.q_slices + k_slices);
+  dim3 grid(a.s.total_qb > a.s.total_kb ? a.s.total_qb : a.s.total_kb, a.q_slices + k_slices);
   if (e4m3)
     pool_kernel<true><<<grid, kPoolThreads, 0, stream>>>(a);
   else

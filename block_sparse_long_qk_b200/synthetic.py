@@ -1,6 +1,6 @@
 """Seeded synthetic workloads for block-sparse causal prefill attention.
 
-This module draws the random inputs that the five workloads are described with and casts
+This module draws the random inputs that the six workloads are described with and casts
 them to the storage types the kernels read (bf16, or e4m3 with per-head absmax scales).
 It holds none of the method's own arithmetic (no pooling, scoring, thresholding or
 attention), so it can feed both the CUDA path and the fp64 oracle without coupling them.
@@ -22,6 +22,11 @@ summary section 4):
 * ``paged``    8 requests, lengths uniform in [4096, 65536], each drawn with the
                ``llama128k`` recipe under its own seed; K/V stored in 64-token pages
                whose physical order is a seeded random permutation.
+* ``chunked``  chunked / prefix-cached prefill in a continuous-batching step: 8 requests
+               with KV lengths uniform in [4096, 131072] (``llama128k`` recipe, 64-token
+               pages as ``paged``); request b prefills only its last q_len_b positions,
+               q_len_b uniform in [1, min(kv_len_b, 16384)], the rest being its cached
+               prefix. Q holds the chunk rows only (drawn for those positions alone).
 
 The vertical, slash (diagonal band) and spatially contiguous patterns these stand in
 for are the ones pattern discovery targets ("FlashPrefill: Instantaneous Pattern
@@ -61,6 +66,8 @@ class Workload:
     dtype: str = "bf16"       # storage type of Q/K/V: "bf16" or "e4m3"
     structure: str = "iid"    # "iid", "vertical" or "band"
     page_size: int = 0        # 0: contiguous K/V; else paged K/V cache with this page size
+    q_lens: tuple | None = None  # chunked prefill: queries per request (the last q_len
+                                 # positions); None = every position is a query
 
     @property
     def total_tokens(self) -> int:
@@ -76,6 +83,13 @@ def paged_lengths(seed: int, n: int = 8, lo: int = 4096, hi: int = 65536) -> tup
     return tuple(int(x) for x in rng.integers(lo, hi + 1, size=n))
 
 
+def chunk_lengths(seed: int, seqlens, cap: int = 16384) -> tuple:
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 78])))
+    return tuple(int(rng.integers(1, min(L, cap) + 1)) for L in seqlens)
+
+
+_CHUNKED_KV = paged_lengths(1240, 8, 4096, 131072)
+
 WORKLOADS = {
     "tiny": Workload("tiny", (2048,), 4, 4, 64, 64, structure="iid"),
     "llama32k": Workload("llama32k", (32768,), 32, 8, 128, 128, structure="vertical"),
@@ -84,10 +98,12 @@ WORKLOADS = {
                          structure="band"),
     "paged": Workload("paged", paged_lengths(1234 + 5), 32, 8, 128, 128, structure="band",
                       page_size=64),
+    "chunked": Workload("chunked", _CHUNKED_KV, 32, 8, 128, 128, structure="band",
+                        page_size=64, q_lens=chunk_lengths(1240, _CHUNKED_KV)),
 }
 
 DEFAULT_SEEDS = {"tiny": 1235, "llama32k": 1236, "llama128k": 1237, "fp8_128k": 1237,
-                 "paged": 1239}
+                 "paged": 1239, "chunked": 1240}
 
 
 def _normal(seed_seq: np.random.SeedSequence, shape) -> np.ndarray:
@@ -117,11 +133,12 @@ def _ar1(seed_seq, T: int, ncomp: int, tau: float) -> np.ndarray:
     return lfilter([1.0], [1.0, -rho], e, axis=0).astype(np.float32)
 
 
-def _one_sequence(w: Workload, L: int, seed_seq: np.random.SeedSequence):
-    """Float32 Q [L,Hq,d], K [L,Hkv,d], V [L,Hkv,d] for one request."""
+def _one_sequence(w: Workload, L: int, seed_seq: np.random.SeedSequence, p0: int = 0):
+    """Float32 Q [L-p0,Hq,d] (positions p0 .. L-1), K [L,Hkv,d], V [L,Hkv,d] for one
+    request."""
     s_q, s_k, s_v, s_u, s_pos, s_band = seed_seq.spawn(6)
     Hq, Hkv, d = w.Hq, w.Hkv, w.d
-    q = _normal(s_q, (L, Hq, d))
+    q = _normal(s_q, (L - p0, Hq, d))
     k = _normal(s_k, (L, Hkv, d))
     v = _normal(s_v, (L, Hkv, d))
     if w.structure == "iid":
@@ -141,7 +158,7 @@ def _one_sequence(w: Workload, L: int, seed_seq: np.random.SeedSequence):
         for g in range(Hkv):
             wg = _ar1(band_seeds[g], L, d, BAND_CORR_TOKENS) * np.float32(BAND_AMPLITUDE)
             k[:, g, :] += wg
-            q[:, g * G:(g + 1) * G, :] += wg[:, None, :]
+            q[:, g * G:(g + 1) * G, :] += wg[p0:, None, :]
     return q, k, v
 
 
@@ -163,13 +180,14 @@ class Inputs:
     q: torch.Tensor
     k: torch.Tensor
     v: torch.Tensor
-    cu_seqlens: torch.Tensor          # int32 [B+1]
+    cu_seqlens: torch.Tensor          # int32 [B+1] key rows (and query rows unless chunked)
     q_scale: torch.Tensor | None = None
     k_scale: torch.Tensor | None = None
     v_scale: torch.Tensor | None = None
     k_cache: torch.Tensor | None = None   # [num_pages, page, Hkv, d] (paged workloads)
     v_cache: torch.Tensor | None = None
     page_table: torch.Tensor | None = None  # int32 [B, max_pages]
+    cu_q: torch.Tensor | None = None  # int32 [B+1] query rows of a chunked workload
 
     def codes_f32(self, which: str) -> np.ndarray:
         """The stored values (bf16 values or e4m3 codes) as float32 -- exact for both
@@ -181,19 +199,27 @@ class Inputs:
         return None if sc is None else sc.double().numpy()
 
 
-def make_inputs(name_or_w, seed: int | None = None, seqlens=None) -> Inputs:
-    """Draw one workload's inputs on the host. ``seqlens`` overrides the request lengths
-    (smaller parity cases keep the recipe and shrink the sizes)."""
+def make_inputs(name_or_w, seed: int | None = None, seqlens=None, q_lens=None) -> Inputs:
+    """Draw one workload's inputs on the host. ``seqlens`` (and ``q_lens``) override the
+    request lengths (smaller parity cases keep the recipe and shrink the sizes). A chunked
+    workload draws K/V for every position and Q for the last q_len positions of each
+    request."""
     w = WORKLOADS[name_or_w] if isinstance(name_or_w, str) else name_or_w
     if seqlens is not None:
         w = dataclasses.replace(w, seqlens=tuple(int(s) for s in seqlens))
+    if q_lens is not None:
+        w = dataclasses.replace(w, q_lens=tuple(int(s) for s in q_lens))
+    if w.q_lens is not None and (len(w.q_lens) != w.batch or
+                                 any(not 0 <= n <= L for n, L in zip(w.q_lens, w.seqlens))):
+        raise ValueError("q_lens needs one entry per request, each in [0, kv_len]")
     if seed is None:
         seed = DEFAULT_SEEDS.get(w.name, 1234)
     root = np.random.SeedSequence(seed)
     req_seeds = root.spawn(w.batch + 1)
     qs, ks, vs = [], [], []
     for b, L in enumerate(w.seqlens):
-        q, k, v = _one_sequence(w, L, req_seeds[b])
+        p0 = L - w.q_lens[b] if w.q_lens is not None else 0
+        q, k, v = _one_sequence(w, L, req_seeds[b], p0)
         qs.append(q)
         ks.append(k)
         vs.append(v)
@@ -204,6 +230,9 @@ def make_inputs(name_or_w, seed: int | None = None, seqlens=None) -> Inputs:
     cu = torch.zeros(w.batch + 1, dtype=torch.int32)
     cu[1:] = torch.cumsum(torch.tensor(w.seqlens, dtype=torch.int64), 0).to(torch.int32)
     inp = Inputs(w, q, k, v, cu)
+    if w.q_lens is not None:
+        inp.cu_q = torch.zeros(w.batch + 1, dtype=torch.int32)
+        inp.cu_q[1:] = torch.cumsum(torch.tensor(w.q_lens, dtype=torch.int64), 0).to(torch.int32)
     if w.dtype == "e4m3":
         inp.q, inp.q_scale = quantize_e4m3(q)
         inp.k, inp.k_scale = quantize_e4m3(k)

@@ -15,6 +15,8 @@
  *                            Block-Sparse Prefill Attention for Long-Context LLM Serving",
  *                            Abstract)
  *   fp_sparse_prefill_attn_paged   the same with K/V read through a page table
+ *   fp_*_chunked             the three stages for chunked / prefix-cached prefill, where each
+ *                            request's queries are the last q_len of its kv_len positions
  *
  * Conventions for every call:
  *  - Every pointer argument is a DEVICE pointer unless its comment says "host". The caller
@@ -162,6 +164,80 @@ int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void*
                                  int max_pages, int num_pages, float scale,
                                  const int32_t* kv_cnt, const int32_t* kv_idx, void* out,
                                  float* lse, void* workspace, void* stream);
+
+/*
+ * Chunked (prefix-cached) prefill. "FlashPrefill V2: Block-Sparse Prefill Attention for
+ * Long-Context LLM Serving", Abstract: the kernels serve as the attention backend of a
+ * continuous-batching engine with a paged KV cache. In such an engine a request's prefill may
+ * run in chunks, or start after a cached prefix: its new queries are then the LAST q_len of
+ * its kv_len positions, and they attend to the cached keys as well as to each other. These
+ * three calls take the stages above to that case; with q_len = kv_len for every request they
+ * compute exactly what the plain calls compute.
+ *
+ * Varlen description (all four arrays int32 [batch + 1], ascending from 0, device memory):
+ *  - cu_k: key rows. Request b holds L_b = cu_k[b+1] - cu_k[b] keys (positions 0 .. L_b - 1);
+ *    total_k = cu_k[batch].
+ *  - cu_q: query rows. Request b holds n_b = cu_q[b+1] - cu_q[b] <= L_b queries, at positions
+ *    P0_b = L_b - n_b .. L_b - 1 (causality aligned at the bottom right: query position p sees
+ *    keys 0 .. p); total_q = cu_q[batch]. n_b = 0 is allowed (the request has no query block).
+ *  - cu_kblocks: ceil(L_b / block) KV blocks per request (blocks of absolute positions,
+ *    restarting at each request); total_kblocks = cu_kblocks[batch].
+ *  - cu_qblocks: the query blocks of request b are the absolute blocks I = floor(P0_b / block)
+ *    .. ceil(L_b / block) - 1, so cu_qblocks[b+1] - cu_qblocks[b] = ceil(L_b / block) -
+ *    floor(P0_b / block) (0 when n_b = 0); total_qblocks = cu_qblocks[batch]. The first query
+ *    block of a request may hold fewer than `block` queries (positions before P0_b belong to
+ *    the prefix); the last one may too (positions past L_b).
+ * Every array is indexed by global query block Ig (0 .. total_qblocks - 1) where the plain
+ * calls use global block Ig, and key-side arrays by global KV block: q_pool [Hq,
+ * total_qblocks, d], k_pool [Hkv, total_kblocks, d], k_pool_split bf16 [2, Hkv, total_kblocks,
+ * d] (or NULL), mask_bits uint32 [Hq, total_qblocks, ceil(max_kblocks / 32)] (or NULL), kv_cnt
+ * [Hq, total_qblocks], kv_idx [Hq, total_qblocks, max_kblocks] with max_kblocks >= the largest
+ * ceil(L_b / block). Kept-block indices are request-local absolute KV blocks J = 0 .. I.
+ * The host does not read the prefix sums: they must agree with the totals and with each other
+ * as stated here (as cu_seqlens / cu_blocks must for the plain calls).
+ *
+ * fp_pool_qk_chunked: the pooled mean of query block I of request b runs over the queries it
+ * holds (positions max(P0_b, I * block) .. min(L_b, (I + 1) * block) - 1); KV block J averages
+ * the keys at positions J * block .. min(L_b, (J + 1) * block) - 1. K is contiguous [total_k,
+ * Hkv, d] or, with k_page_table != NULL, the cache [num_pages, page_size, Hkv, d] read through
+ * page_table int32 [batch, max_pages] (same rules as fp_pool_qk). Q is contiguous [total_q,
+ * Hq, d].
+ * fp_build_block_mask_chunked: row Ig (absolute block I of request b) scores KV blocks J = 0 ..
+ * I of request b, with the same threshold, flags and outputs as fp_build_block_mask. `block` is
+ * needed to place query blocks (64 or 128).
+ * fp_sparse_prefill_attn_chunked: out [total_q, Hq, d] bf16 and lse [Hq, total_q] (or NULL) for
+ * the queries only. K and V are contiguous [total_k, Hkv, d] (page_table NULL) or caches read
+ * through page_table (same rules as fp_sparse_prefill_attn_paged). Errors as fp_pool_qk,
+ * fp_build_block_mask and fp_sparse_prefill_attn respectively.
+ */
+int fp_pool_qk_chunked(const void* q, const void* k, int dtype, const float* q_scale,
+                       const float* k_scale, const int32_t* cu_q, const int32_t* cu_qblocks,
+                       const int32_t* cu_k, const int32_t* cu_kblocks, int batch, int total_q,
+                       int total_k, int total_qblocks, int total_kblocks, int Hq, int Hkv,
+                       int d, int block, const int32_t* k_page_table, int page_size,
+                       int max_pages, int num_pages, float* q_pool, float* k_pool,
+                       void* k_pool_split, void* stream);
+
+int fp_build_block_mask_chunked(const float* q_pool, const float* k_pool,
+                                const void* k_pool_split, const int32_t* cu_q,
+                                const int32_t* cu_qblocks, const int32_t* cu_k,
+                                const int32_t* cu_kblocks, int batch, int total_qblocks,
+                                int total_kblocks, int max_kblocks, int Hq, int Hkv, int d,
+                                int block, float alpha, float scale, int flags,
+                                uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx,
+                                void* stream);
+
+int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, int dtype,
+                                   const float* q_scale, const float* k_scale,
+                                   const float* v_scale, const int32_t* cu_q,
+                                   const int32_t* cu_qblocks, const int32_t* cu_k,
+                                   const int32_t* cu_kblocks, int batch, int total_q,
+                                   int total_k, int total_qblocks, int total_kblocks,
+                                   int max_kblocks, int Hq, int Hkv, int d, int block,
+                                   const int32_t* page_table, int page_size, int max_pages,
+                                   int num_pages, float scale, const int32_t* kv_cnt,
+                                   const int32_t* kv_idx, void* out, float* lse,
+                                   void* workspace, void* stream);
 
 /*
  * fp_pool_qk followed by fp_build_block_mask, for callers that cannot allocate device memory.

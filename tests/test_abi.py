@@ -57,3 +57,51 @@ def test_mask_rejects_alpha_out_of_range():
                                  16, None)
     assert rc == -1
     assert b"alpha" in lib.fp_last_error_string()
+
+
+def test_chunked_batch_layout():
+    """Host-side prefix sums of a chunked batch (query blocks start at floor(P0 / block))."""
+    cb = fp.ChunkedBatch.make((1000, 0, 37, 641, 1), (1000, 700, 300, 1500, 129), 128, "cpu")
+    # query blocks: [0, 8), none, [2, 3), [6, 12), [1, 2)
+    assert cb.cu_qblocks.tolist() == [0, 8, 8, 9, 15, 16]
+    assert cb.cu_kblocks.tolist() == [0, 8, 14, 17, 29, 31]
+    assert (cb.total_q, cb.total_k, cb.max_kblocks) == (1679, 3629, 12)
+
+
+def _bad_chunked_attn(**over):
+    """A well-formed chunked attention call with fake pointers (host validation only)."""
+    a = dict(q=16, k=16, v=16, dtype=0, qs=None, ks=None, vs=None, cq=16, cqb=16, ck=16, ckb=16,
+             batch=2, Tq=300, Tk=1000, tqb=4, tkb=9, mkb=5, Hq=8, Hkv=2, d=128, block=128,
+             pt=None, ps=0, mp=0, npg=0, scale=0.1, cnt=16, idx=16, out=16, lse=None, ws=256,
+             stream=None)
+    a.update(over)
+    return fp.library().fp_sparse_prefill_attn_chunked(*a.values())
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(cq=None), -1),             # chunked calls need every prefix-sum array
+    (dict(ckb=None), -1),
+    (dict(Tq=1001), -1),             # more queries than keys
+    (dict(tqb=10), -1),              # more query blocks than key blocks
+    (dict(mkb=0), -1),               # no room for a kept-block list
+    (dict(block=96), -2),
+    (dict(pt=16, ps=48), -1),        # page size not dividing the block
+    (dict(dtype=1, qs=16, ks=16, vs=16, d=64), -2),   # e4m3 needs d = 128
+])
+def test_chunked_attention_rejects_bad_arguments(over, code):
+    assert _bad_chunked_attn(**over) == code
+    assert fp.library().fp_last_error_string()
+
+
+def test_chunked_mask_and_pool_reject_bad_arguments():
+    lib = fp.library()
+    # mask: block size is needed to place query blocks
+    rc = lib.fp_build_block_mask_chunked(16, 16, None, 16, 16, 16, 16, 2, 4, 9, 5, 8, 2, 128, 96,
+                                         0.1, 0.1, 3, None, 16, 16, None)
+    assert rc == -2
+    rc = lib.fp_build_block_mask_chunked(16, 16, None, None, 16, 16, 16, 2, 4, 9, 5, 8, 2, 128,
+                                         128, 0.1, 0.1, 3, None, 16, 16, None)
+    assert rc == -1
+    rc = lib.fp_pool_qk_chunked(16, 16, 0, None, None, 16, 16, 16, 16, 2, 1001, 1000, 4, 9, 8, 2,
+                                128, 128, None, 0, 0, 0, 16, 16, None, None)
+    assert rc == -1 and b"total_q" in lib.fp_last_error_string()

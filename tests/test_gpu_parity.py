@@ -263,16 +263,23 @@ def _full_size(name, cuda_device, n_rows=48):
     w = inp.workload
     run = OracleRun(inp, w.alpha)
     q, k, v, sc = device_inputs(inp, cuda_device)
-    b = _batch(inp, cuda_device)
     paged = _paged(inp, cuda_device)
-    qp, kp = fp.pool_qk(q, k, w.block, batch=b, q_scale=sc["q_scale"], k_scale=sc["k_scale"],
-                        paged=paged)
-    bits, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b)
     kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"])
-    if paged is not None:
-        out, _ = fp.sparse_prefill_attn_paged(q, paged, cnt, idx, b, **kw)
+    if run.chunked:
+        cb = fp.ChunkedBatch.make(w.q_lens, w.seqlens, w.block, cuda_device)
+        qp, kp = fp.pool_qk_chunked(q, k, cb, q_scale=sc["q_scale"], k_scale=sc["k_scale"],
+                                    paged=paged)
+        bits, cnt, idx = fp.build_block_mask_chunked(qp, kp, cb, w.alpha)
+        out, _ = fp.sparse_prefill_attn_chunked(q, k, v, cnt, idx, cb, paged=paged, **kw)
     else:
-        out, _ = fp.sparse_prefill_attn(q, k, v, cnt, idx, w.block, batch=b, **kw)
+        b = _batch(inp, cuda_device)
+        qp, kp = fp.pool_qk(q, k, w.block, batch=b, q_scale=sc["q_scale"],
+                            k_scale=sc["k_scale"], paged=paged)
+        bits, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b)
+        if paged is not None:
+            out, _ = fp.sparse_prefill_attn_paged(q, paged, cnt, idx, b, **kw)
+        else:
+            out, _ = fp.sparse_prefill_attn(q, k, v, cnt, idx, w.block, batch=b, **kw)
     fp.check_status(cuda_device)
     gk = bits_to_keeps(bits, run)
     bad, ex, tot = mask_mismatches(gk, run)
@@ -280,14 +287,15 @@ def _full_size(name, cuda_device, n_rows=48):
     # sampled (head, query block) rows whose GPU and oracle masks agree
     rng = np.random.default_rng(11)
     rows = []
+    nrows = run.qoff[-1]
     while len(rows) < n_rows:
         h = int(rng.integers(w.Hq))
-        Ig = int(rng.integers(run.off[-1]))
-        r = int(np.searchsorted(run.off, Ig, side="right") - 1)
-        I = Ig - run.off[r]
-        if np.array_equal(gk[r][h, I], run.keeps[r][h, I]):
+        Ig = int(rng.integers(nrows))
+        r = int(np.searchsorted(run.qoff, Ig, side="right") - 1)
+        i = Ig - run.qoff[r]
+        if np.array_equal(gk[r][h, i], run.keeps[r][h, i]):
             rows.append((h, Ig))
-    rows.append((0, run.off[-1] - 1))
+    rows.append((0, nrows - 1))
     ref, _ = run.attention(rows=rows)
     amax, rel = attn_errors(out, ref)
     tol = TOL[w.dtype]
@@ -295,6 +303,6 @@ def _full_size(name, cuda_device, n_rows=48):
     return run
 
 
-@pytest.mark.parametrize("name", ["llama32k", "llama128k", "fp8_128k", "paged"])
+@pytest.mark.parametrize("name", ["llama32k", "llama128k", "fp8_128k", "paged", "chunked"])
 def test_full_size_workloads(name, cuda_device):
     _full_size(name, cuda_device)

@@ -52,3 +52,26 @@ def test_vertical_stripes_planted():
     # 64 planted rows stand out by the 3u shift: norm ~ sqrt(11.3 + 9) = 4.5 against a
     # base norm ~ sqrt(128 / sqrt(128)) = 3.4 (averaged over the 8 KV heads)
     assert int((norms > norms.median() + 0.6).sum()) == 64
+
+
+def test_chunked_queries_are_the_last_positions():
+    w = S.WORKLOADS["chunked"]
+    assert len(w.q_lens) == w.batch and all(1 <= n <= min(L, 16384)
+                                            for n, L in zip(w.q_lens, w.seqlens))
+    small = S.make_inputs(w, seqlens=(300, 700, 5), q_lens=(100, 0, 5))
+    assert small.q.shape == (105, w.Hq, w.d) and small.k.shape == (1005, w.Hkv, w.d)
+    assert small.cu_q.tolist() == [0, 100, 100, 105]
+    assert small.cu_seqlens.tolist() == [0, 300, 1000, 1005]
+    # With every position a query, the chunked draw is the plain draw of the same recipe.
+    full = S.make_inputs(w, seqlens=(300, 70), q_lens=(300, 70))
+    plain = S.make_inputs(S.Workload("chunked", (300, 70), w.Hq, w.Hkv, w.d, w.block,
+                                     structure=w.structure, page_size=w.page_size),
+                          seed=S.DEFAULT_SEEDS["chunked"])
+    for n in ("q", "k", "v", "k_cache", "page_table"):
+        assert torch.equal(getattr(full, n), getattr(plain, n)), n
+    try:
+        S.make_inputs(w, seqlens=(10,), q_lens=(11,))
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("q_len > kv_len accepted")
