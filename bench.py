@@ -187,15 +187,16 @@ def work_counts(w, cnt, idx, batch=None):
 
 
 def pool_mask_bytes(w):
+    """(pool kernel bytes, pool + mask bytes): Q and K read once, the fp32 means and the bf16
+    hi / lo split of the pooled keys written by the pool kernel and read by the mask kernel."""
     eb = 1 if w.dtype == "e4m3" else 2
     Tk = w.total_tokens
     Tq = sum(w.q_lens) if w.q_lens is not None else Tk
     nkb = sum((L + w.block - 1) // w.block for L in w.seqlens)
     nqb = len(_query_blocks(w)[0])
-    # Q and K read once; pooled means written (fp32) and read back by the mask kernel, plus the
-    # bf16 hi / lo split of the pooled keys written and read
-    return ((Tq * w.Hq + Tk * w.Hkv) * w.d * eb + 2 * (nqb * w.Hq + nkb * w.Hkv) * w.d * 4
-            + 2 * nkb * w.Hkv * w.d * 4)
+    inputs = (Tq * w.Hq + Tk * w.Hkv) * w.d * eb
+    pooled = (nqb * w.Hq + nkb * w.Hkv) * w.d * 4 + nkb * w.Hkv * w.d * 4
+    return inputs + pooled, inputs + 2 * pooled
 
 
 def cpu_baseline(inp, rows_sample=32, seed=5):
@@ -333,7 +334,7 @@ def run_native(args, world, rank, local):
     pool_ms, mask_ms, attn_ms = (statistics.mean(x) for x in (pool_l, mask_l, attn_l))
 
     alg, executed, density = work_counts(w, cnt, idx)
-    pm_bytes = pool_mask_bytes(w)
+    pool_bytes, pm_bytes = pool_mask_bytes(w)
     peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     if w.dtype == "e4m3":
         peak_t *= 2.0   # e4m3 dense rate = 2x bf16 (nominal ratio); no measured e4m3 peak
@@ -375,7 +376,8 @@ def run_native(args, world, rank, local):
                           "gbs": round(pm_bytes / ((pool_ms + mask_ms) * 1e-3) / 1e9, 1),
                           "frac_hbm": round(pm_bytes / ((pool_ms + mask_ms) * 1e-3) / 1e9 /
                                             peaks["hbm_gbs"], 4),
-                          "pool_frac_hbm": round(pm_bytes / (pool_ms * 1e-3) / 1e9 /
+                          "pool_bytes": pool_bytes,
+                          "pool_frac_hbm": round(pool_bytes / (pool_ms * 1e-3) / 1e9 /
                                                  peaks["hbm_gbs"], 4)},
             "block_density": round(density, 5),
             "attn_tflop": {"algorithmic": round(alg / 1e12, 3),
