@@ -32,7 +32,8 @@ __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_at
            "sparse_prefill_attn_paged", "sparse_prefill", "check_status", "workspace",
            "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "header_symbols",
            "pool_and_mask_noalloc", "k_split_shape", "ChunkedBatch", "pool_qk_chunked",
-           "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked"]
+           "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked",
+           "HostPipeline"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfpsparse.so")
@@ -304,9 +305,9 @@ def sparse_prefill_attn_paged(q, paged: PagedKV, kv_cnt, kv_idx, batch: Batch, *
 
 def sparse_prefill(q, k=None, v=None, alpha=0.1, block=128, *, batch: Batch | None = None,
                    paged: PagedKV | None = None, scale=None, q_scale=None, k_scale=None,
-                   v_scale=None, return_lse=False, flags=FORCE_FIRST | FORCE_DIAG):
+                   v_scale=None, return_lse=False, flags=FORCE_FIRST | FORCE_DIAG, out=None):
     """The whole path: pool -> threshold/mask -> sparse attention. Returns
-    (out, lse or None, kv_cnt, kv_idx)."""
+    (out, lse or None, kv_cnt, kv_idx); ``out`` may be a preallocated bf16 [T, Hq, d]."""
     b = _batch_for(q, block, batch)
     d = q.shape[-1]
     if scale is None:
@@ -322,11 +323,11 @@ def sparse_prefill(q, k=None, v=None, alpha=0.1, block=128, *, batch: Batch | No
     if paged is not None:
         out, lse = sparse_prefill_attn_paged(q, paged, kv_cnt, kv_idx, b, scale=scale,
                                              q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,
-                                             return_lse=return_lse)
+                                             return_lse=return_lse, out=out)
     else:
         out, lse = sparse_prefill_attn(q, k, v, kv_cnt, kv_idx, block, batch=b, scale=scale,
                                        q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,
-                                       return_lse=return_lse)
+                                       return_lse=return_lse, out=out)
     return out, lse, kv_cnt, kv_idx
 
 
@@ -482,7 +483,7 @@ def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
 def sparse_prefill_chunked(q, k, v, cb: ChunkedBatch, alpha=0.1, *,
                            paged: PagedKV | None = None, scale=None, q_scale=None,
                            k_scale=None, v_scale=None, return_lse=False,
-                           flags=FORCE_FIRST | FORCE_DIAG):
+                           flags=FORCE_FIRST | FORCE_DIAG, out=None):
     """The whole path for a chunked batch. Returns (out, lse or None, kv_cnt, kv_idx)."""
     d = q.shape[-1]
     if scale is None:
@@ -496,5 +497,59 @@ def sparse_prefill_chunked(q, k, v, cb: ChunkedBatch, alpha=0.1, *,
                                                  flags=flags, mask_bits=False, k_split=k_split)
     out, lse = sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb, paged=paged, scale=scale,
                                            q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,
-                                           return_lse=return_lse)
+                                           return_lse=return_lse, out=out)
     return out, lse, kv_cnt, kv_idx
+
+
+class HostPipeline:
+    """Runs the path step after step on inputs and outputs in pinned host memory, overlapping
+    each step's host-to-device copies and the previous step's device-to-host copy with the
+    kernels (three CUDA streams: copy-in, compute, copy-out; ``depth`` device buffer sets).
+
+    ``run(*device_inputs, out=device_out)`` enqueues one step on the current stream (e.g. a
+    call of ``sparse_prefill`` with the layer's fixed arguments bound). ``submit`` copies the
+    host inputs in, runs the step and copies its output back into ``host_out``; it returns at
+    once. ``synchronize`` waits for every submitted step. Host tensors must not be changed
+    until the step that reads or writes them has completed."""
+
+    def __init__(self, run, input_like, out_like, device, depth=2):
+        self.run = run
+        self.device = torch.device(device)
+        self.depth = depth
+        self.h2d = torch.cuda.Stream(self.device)
+        self.comp = torch.cuda.Stream(self.device)
+        self.d2h = torch.cuda.Stream(self.device)
+        self.dev_in = [[torch.empty(t.shape, dtype=t.dtype, device=self.device)
+                        for t in input_like] for _ in range(depth)]
+        self.dev_out = [torch.empty(out_like.shape, dtype=out_like.dtype, device=self.device)
+                        for _ in range(depth)]
+        self.in_free = [None] * depth    # compute of the step that last read buffer set i
+        self.out_free = [None] * depth   # copy-out of the step that last wrote buffer set i
+        self.n = 0
+
+    def submit(self, host_inputs, host_out):
+        i = self.n % self.depth
+        self.n += 1
+        ev_in, ev_done, ev_out = (torch.cuda.Event() for _ in range(3))
+        with torch.cuda.stream(self.h2d):
+            if self.in_free[i] is not None:
+                self.h2d.wait_event(self.in_free[i])
+            for d, h in zip(self.dev_in[i], host_inputs):
+                d.copy_(h, non_blocking=True)
+            ev_in.record(self.h2d)
+        with torch.cuda.stream(self.comp):
+            self.comp.wait_event(ev_in)
+            if self.out_free[i] is not None:
+                self.comp.wait_event(self.out_free[i])
+            self.run(*self.dev_in[i], out=self.dev_out[i])
+            ev_done.record(self.comp)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(ev_done)
+            host_out.copy_(self.dev_out[i], non_blocking=True)
+            ev_out.record(self.d2h)
+        self.in_free[i] = ev_done
+        self.out_free[i] = ev_out
+
+    def synchronize(self):
+        for st in (self.h2d, self.comp, self.d2h):
+            st.synchronize()
