@@ -399,15 +399,28 @@ def run_e2e(layer, inp, dev, args, world):
     included."""
     w = layer.w
     hq = inp.q.pin_memory()
-    hk = (inp.k_cache if inp.k_cache is not None else inp.k).pin_memory()
-    hv = (inp.v_cache if inp.v_cache is not None else inp.v).pin_memory()
     houts = [torch.empty(layer.q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     sc = layer.scales
     pt = layer.paged.page_table if layer.paged is not None else None
+    append = layer.cb is not None and layer.paged is not None
+    if append:
+        # Chunked prefill on a paged cache: the cached prefix stays on the device; each step
+        # copies in the chunk's Q, K and V rows and appends K/V to the cache before attention.
+        cu = inp.cu_seqlens.tolist()
+        rows = torch.cat([torch.arange(cu[b] + L - n, cu[b] + L)
+                          for b, (n, L) in enumerate(zip(w.q_lens, w.seqlens))])
+        hk, hv = inp.k[rows].pin_memory(), inp.v[rows].pin_memory()
+    else:
+        hk = (inp.k_cache if inp.k_cache is not None else inp.k).pin_memory()
+        hv = (inp.v_cache if inp.v_cache is not None else inp.v).pin_memory()
 
     def run(q, k, v, out):
-        paged = fp.PagedKV(k, v, pt) if pt is not None else None
         kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"], out=out)
+        if append:
+            fp.append_paged_kv(k, v, layer.cb, layer.paged)
+            fp.sparse_prefill_chunked(q, None, None, layer.cb, w.alpha, paged=layer.paged, **kw)
+            return
+        paged = fp.PagedKV(k, v, pt) if pt is not None else None
         if layer.cb is not None:
             fp.sparse_prefill_chunked(q, k, v, layer.cb, w.alpha, paged=paged, **kw)
         elif paged is not None:
@@ -436,7 +449,9 @@ def run_e2e(layer, inp, dev, args, world):
         hv.numel() * hv.element_size()
     return {"value": round(ms / world, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": houts[0].numel() * houts[0].element_size(), "steps": steps,
-            "pipelined": "copy-in, kernels and copy-out of neighbouring steps overlap"}
+            "pipelined": "copy-in, kernels and copy-out of neighbouring steps overlap",
+            "inputs": ("chunk Q, K, V rows (cached prefix resident in the paged cache; the "
+                       "chunk's K/V appended each step)") if append else "Q, K, V"}
 
 
 def main():

@@ -33,7 +33,7 @@ __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_at
            "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "header_symbols",
            "pool_and_mask_noalloc", "k_split_shape", "ChunkedBatch", "pool_qk_chunked",
            "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked",
-           "HostPipeline"]
+           "HostPipeline", "append_paged_kv"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfpsparse.so")
@@ -67,6 +67,8 @@ _SIGNATURES = {
                                 _i, _i, _p, _i, _i, _i, _p, _p, _p, _p]),
     "fp_build_block_mask_chunked": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
                                          _i, _i, _f, _f, _i, _p, _p, _p, _p]),
+    "fp_append_paged_kv": (_i, [_p, _p, _i, _p, _p, _i, _i, _i, _i, _p, _i, _i, _i, _p, _p, _p,
+                                _p]),
     "fp_sparse_prefill_attn_chunked": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _i, _i,
                                             _i, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _i, _f,
                                             _p, _p, _p, _p, _p, _p]),
@@ -478,6 +480,18 @@ def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
         float(scale), _ptr(kv_cnt), _ptr(kv_idx), _ptr(out), _ptr(lse), _ptr(ws),
         _stream(q.device)))
     return out, lse
+
+
+def append_paged_kv(k_new, v_new, cb: ChunkedBatch, paged: PagedKV, *, ws=None):
+    """Writes the chunk's new K and V rows [total_q, Hkv, d] into the paged caches at their
+    absolute positions (before the chunked prefill reads them)."""
+    T, Hkv, d = k_new.shape
+    ws = workspace(k_new.device) if ws is None else ws
+    pt = paged.page_table
+    _check(library().fp_append_paged_kv(
+        _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(cb.cu_q), _ptr(cb.cu_k), cb.size, T,
+        Hkv, d, _ptr(pt), paged.page_size, pt.shape[1], paged.k_cache.shape[0],
+        _ptr(paged.k_cache), _ptr(paged.v_cache), _ptr(ws), _stream(k_new.device)))
 
 
 def sparse_prefill_chunked(q, k, v, cb: ChunkedBatch, alpha=0.1, *,

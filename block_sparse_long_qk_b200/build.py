@@ -15,7 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfpsparse.so")
-SOURCES = ["api.cu", "pool.cu", "mask.cu", "mask_tc.cu", "attn.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "pool.cu", "mask.cu", "mask_tc.cu", "attn.cu", "noalloc.cu", "append.cu"]
 HEADERS = ["fp_common.cuh", "fp_launch.h", os.path.join("..", "..", "include", "fpsparse.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -428,6 +428,43 @@ int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, 
                    kv_idx, out, lse, workspace, stream);
 }
 
+int fp_append_paged_kv(const void* k_new, const void* v_new, int dtype, const int32_t* cu_q,
+                       const int32_t* cu_k, int batch, int total_q, int Hkv, int d,
+                       const int32_t* page_table, int page_size, int max_pages, int num_pages,
+                       void* k_cache, void* v_cache, void* workspace, void* stream) {
+  g_err.clear();
+  if (dtype != FP_DTYPE_BF16 && dtype != FP_DTYPE_E4M3)
+    return fail(FP_ERR_INVALID_ARG, "dtype %d is neither FP_DTYPE_BF16 nor FP_DTYPE_E4M3", dtype);
+  if (d != 64 && d != 128) return fail(FP_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  if (batch < 1 || Hkv < 1 || total_q < 0)
+    return fail(FP_ERR_INVALID_ARG, "batch and Hkv must be >= 1, total_q >= 0");
+  if (!k_new || !v_new || !cu_q || !cu_k || !page_table || !k_cache || !v_cache || !workspace)
+    return fail(FP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(FP_ERR_INVALID_ARG, "K/V rows and caches must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (page_size < 1 || max_pages < 1 || num_pages < 1)
+    return fail(FP_ERR_INVALID_ARG, "page_size, max_pages and num_pages must be >= 1");
+  fp::AppendArgs a{};
+  a.k_new = static_cast<const uint8_t*>(k_new);
+  a.v_new = static_cast<const uint8_t*>(v_new);
+  a.k_cache = static_cast<uint8_t*>(k_cache);
+  a.v_cache = static_cast<uint8_t*>(v_cache);
+  a.page_table = page_table;
+  a.status = static_cast<uint32_t*>(workspace);
+  a.s.cu_q = cu_q;
+  a.s.cu_k = cu_k;
+  a.s.batch = batch;
+  a.s.total_q = total_q;
+  a.row_bytes = Hkv * d * (dtype == FP_DTYPE_E4M3 ? 1 : 2);
+  a.page_size = page_size;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  cudaError_t e = fp::launch_append(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP_OK : cuda_fail(e, "append kernel launch");
+}
+
 int fp_debug_skip_k_load(int union_block) {
   g_err.clear();
   if (union_block < 0) return fail(FP_ERR_INVALID_ARG, "union block index must be >= 0");

@@ -70,6 +70,18 @@ struct AttnArgs {
   float scale_log2;                     // softmax scale * log2(e)
 };
 
+struct AppendArgs {
+  const uint8_t* k_new;  // [total_q, Hkv, d] rows of the new chunk
+  const uint8_t* v_new;
+  uint8_t* k_cache;      // [num_pages, page_size, Hkv, d]
+  uint8_t* v_cache;
+  const int32_t* page_table;  // [batch, max_pages]
+  uint32_t* status;
+  Seqs s;
+  int row_bytes;  // Hkv * d * element size
+  int page_size, max_pages, num_pages;
+};
+
 struct AttnLaunch {
   const void *q, *k, *v;
   bool e4m3, paged;
@@ -84,6 +96,7 @@ int mask_blocks_per_cta(int G, int d, int max_kb);
 bool mask_tc_supported(int G, int d);   // tensor-core scores (mask_tc.cu) apply
 cudaError_t launch_mask_tc(const MaskArgs& a, cudaStream_t stream);
 cudaError_t launch_attn(const AttnArgs& a, const AttnLaunch& L, int block, cudaStream_t stream);
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 
 // cuTensorMapEncodeTiled, looked up once through the runtime (no link against libcuda).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -17,6 +17,7 @@
  *   fp_sparse_prefill_attn_paged   the same with K/V read through a page table
  *   fp_*_chunked             the three stages for chunked / prefix-cached prefill, where each
  *                            request's queries are the last q_len of its kv_len positions
+ *   fp_append_paged_kv       writes a chunk's new K/V rows into the paged cache first
  *
  * Conventions for every call:
  *  - Every pointer argument is a DEVICE pointer unless its comment says "host". The caller
@@ -238,6 +239,26 @@ int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, 
                                    int num_pages, float scale, const int32_t* kv_cnt,
                                    const int32_t* kv_idx, void* out, float* lse,
                                    void* workspace, void* stream);
+
+/*
+ * Chunked prefill, the step before the three stages: writes the new chunk's K and V rows into
+ * the paged KV cache ("FlashPrefill V2: Block-Sparse Prefill Attention for Long-Context LLM
+ * Serving", Abstract: paged KV cache and continuous batching). Row t of request b (cu_q[b] <=
+ * t < cu_q[b+1]) holds absolute position p = L_b - n_b + (t - cu_q[b]), with L_b = cu_k[b+1] -
+ * cu_k[b] the request's key count after the append and n_b its new rows (the same description
+ * as the fp_*_chunked calls); it is copied bit for bit to slot p % page_size of page
+ * page_table[b][p / page_size] of k_cache and v_cache [num_pages, page_size, Hkv, d].
+ * k_new, v_new  [total_q, Hkv, d], bf16 or e4m3 codes (dtype), 16-byte aligned
+ * workspace     as for the attention calls; a page-table entry outside [0, num_pages) or a
+ *               position past max_pages pages skips that row and records FP_ERR_BAD_INDEX
+ *               (read with fp_check_status).
+ * Supported: d in {64, 128}. Rows of different calls may target the same slots only if the
+ * calls are ordered on one stream.
+ */
+int fp_append_paged_kv(const void* k_new, const void* v_new, int dtype, const int32_t* cu_q,
+                       const int32_t* cu_k, int batch, int total_q, int Hkv, int d,
+                       const int32_t* page_table, int page_size, int max_pages, int num_pages,
+                       void* k_cache, void* v_cache, void* workspace, void* stream);
 
 /*
  * fp_pool_qk followed by fp_build_block_mask, for callers that cannot allocate device memory.

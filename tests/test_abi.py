@@ -105,3 +105,16 @@ def test_chunked_mask_and_pool_reject_bad_arguments():
     rc = lib.fp_pool_qk_chunked(16, 16, 0, None, None, 16, 16, 16, 16, 2, 1001, 1000, 4, 9, 8, 2,
                                 128, 128, None, 0, 0, 0, 16, 16, None, None)
     assert rc == -1 and b"total_q" in lib.fp_last_error_string()
+
+
+def test_append_rejects_bad_arguments():
+    lib = fp.library()
+    args = [16, 16, 0, 16, 16, 2, 300, 2, 128, 16, 64, 8, 40, 16, 16, 256, None]
+    bad_d = list(args); bad_d[8] = 96
+    assert lib.fp_append_paged_kv(*bad_d) == -2
+    null_pt = list(args); null_pt[9] = None
+    assert lib.fp_append_paged_kv(*null_pt) == -1
+    bad_page = list(args); bad_page[10] = 0
+    assert lib.fp_append_paged_kv(*bad_page) == -1
+    misaligned = list(args); misaligned[13] = 8
+    assert lib.fp_append_paged_kv(*misaligned) == -1

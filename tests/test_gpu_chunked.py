@@ -173,3 +173,62 @@ def test_chunked_argument_errors(cuda_device):
     assert e.value.code == -1
     with pytest.raises(ValueError):
         fp.ChunkedBatch.make((11,), (10,), 128, cuda_device)
+
+
+def _chunk_rows(inp):
+    """Host rows of K and V at each request's new (chunk) positions, in request order."""
+    w = inp.workload
+    cu = inp.cu_seqlens.tolist()
+    idx = torch.cat([torch.arange(cu[b] + L - n, cu[b] + L)
+                     for b, (n, L) in enumerate(zip(w.q_lens, w.seqlens))])
+    return inp.k[idx].contiguous(), inp.v[idx].contiguous()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_append_writes_chunk_rows_into_the_paged_cache(dtype, cuda_device):
+    """The append kernel writes the chunk's K/V rows exactly where the full cache has them,
+    and nothing else; the chunked prefill on the appended cache equals the one on the full
+    cache bit for bit."""
+    w = dataclasses.replace(BASE, page_size=64, dtype=dtype)
+    inp = S.make_inputs(w, seed=12, seqlens=(1000, 700, 300, 129), q_lens=(333, 700, 65, 1))
+    w = inp.workload
+    cb = _cb(inp, cuda_device)
+    full = _paged(inp, cuda_device)
+    # a cache holding the prefixes only: every chunk slot cleared
+    k_cache, v_cache = full.k_cache.clone(), full.v_cache.clone()
+    P = w.page_size
+    for b, (n, L) in enumerate(zip(w.q_lens, w.seqlens)):
+        for p in range(L - n, L):
+            page = int(inp.page_table[b, p // P])
+            k_cache.view(torch.uint8)[page, p % P].zero_()
+            v_cache.view(torch.uint8)[page, p % P].zero_()
+    kn, vn = _chunk_rows(inp)
+    cache = fp.PagedKV(k_cache, v_cache, full.page_table)
+    fp.append_paged_kv(kn.to(cuda_device), vn.to(cuda_device), cb, cache)
+    fp.check_status(cuda_device)
+    assert torch.equal(k_cache.view(torch.uint8), full.k_cache.view(torch.uint8))
+    assert torch.equal(v_cache.view(torch.uint8), full.v_cache.view(torch.uint8))
+    q, _, _, sc = device_inputs(inp, cuda_device)
+    kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"])
+    out_a, _, _, _ = fp.sparse_prefill_chunked(q, None, None, cb, 0.5, paged=cache, **kw)
+    out_b, _, _, _ = fp.sparse_prefill_chunked(q, None, None, cb, 0.5, paged=full, **kw)
+    fp.check_status(cuda_device)
+    assert torch.equal(out_a, out_b)
+
+
+def test_append_reports_a_bad_page_entry(cuda_device):
+    w = dataclasses.replace(BASE, page_size=64)
+    inp = S.make_inputs(w, seed=13, seqlens=(300,), q_lens=(100,))
+    cb = _cb(inp, cuda_device)
+    full = _paged(inp, cuda_device)
+    pt = full.page_table.clone()
+    pt[0, 299 // 64] = 10 ** 6          # the page of the last rows points past the cache
+    kn, vn = _chunk_rows(inp)
+    before = full.k_cache.clone()
+    fp.append_paged_kv(kn.to(cuda_device), vn.to(cuda_device), cb,
+                       fp.PagedKV(full.k_cache, full.v_cache, pt))
+    with pytest.raises(fp.FpError) as e:
+        fp.check_status(cuda_device)
+    assert e.value.code == -5
+    # rows whose page is valid were written (with the values they already had)
+    assert torch.equal(full.k_cache, before)
