@@ -146,7 +146,10 @@ def block_scores(q_pool, k_pool, cu_seqlens, block, scale, cu_k=None):
 
 
 def _row_softmax(s):
-    """Softmax over the last axis of a score array whose masked entries are -inf."""
+    """Softmax over the last axis of a score array whose masked entries are -inf. A request
+    without tokens has no blocks: its (empty) array is returned as it is."""
+    if s.shape[-1] == 0:
+        return s.copy()
     m = s.max(axis=-1, keepdims=True)
     e = np.exp(s - m)
     return e / e.sum(axis=-1, keepdims=True)
@@ -157,9 +160,11 @@ def block_keep(scores, alpha, force_first=True, force_diag=True, row0=0):
 
     p = softmax over the causal pooled row; keep J iff p[J] >= alpha * max_J p, plus the
     diagonal block J = I and the first block J = 0 when forced."""
+    nq, n = scores.shape[-2:]
+    if n == 0:
+        return np.zeros(scores.shape, dtype=bool)
     p = _row_softmax(scores)
     keep = p >= alpha * p.max(axis=-1, keepdims=True)
-    nq, n = scores.shape[-2:]
     rows = row0 + np.arange(nq)
     causal = np.arange(n)[None, :] <= rows[:, None]
     keep &= causal[None]
@@ -174,6 +179,8 @@ def keep_ratio(scores):
     """p[J] / max p over each causal row (float64; 0 above the diagonal). A block whose
     ratio lies within a relative 1e-3 of alpha sits on the threshold, where fp32 and fp64
     may legitimately decide differently."""
+    if scores.shape[-1] == 0:
+        return scores.copy()
     p = _row_softmax(scores)
     return p / p.max(axis=-1, keepdims=True)
 

@@ -118,3 +118,15 @@ def test_append_rejects_bad_arguments():
     assert lib.fp_append_paged_kv(*bad_page) == -1
     misaligned = list(args); misaligned[13] = 8
     assert lib.fp_append_paged_kv(*misaligned) == -1
+
+
+def test_empty_inputs_return_ok_without_launching():
+    """No tokens: every stage returns FP_OK before any CUDA call (this runs without a GPU)."""
+    lib = fp.library()
+    assert lib.fp_pool_qk(16, 16, 0, None, None, None, None, 1, 0, 0, 8, 2, 128, 128, None, 0, 0,
+                          0, 16, 16, None, None) == 0
+    assert lib.fp_build_block_mask(16, 16, None, None, 1, 0, 0, 8, 2, 128, 0.1, 0.1, 3, None, 16,
+                                   16, None) == 0
+    assert _bad_attn(T=0, tb=0, mb=0) == 0
+    assert lib.fp_append_paged_kv(16, 16, 0, 16, 16, 1, 0, 2, 128, 16, 64, 1, 1, 16, 16, 256,
+                                  None) == 0

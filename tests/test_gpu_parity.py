@@ -50,6 +50,11 @@ def _case(name):
         "gqa8": (dataclasses.replace(base, Hq=16, Hkv=2, structure="iid"), (3000,), 0.5),
         # group of 3: the fp32 FFMA mask kernel and single-tile attention CTAs
         "gqa3_ffma": (dataclasses.replace(base, Hq=6, Hkv=2, structure="iid"), (1500,), 0.5),
+        # a request without tokens between two others (no blocks, no rows)
+        "varlen_empty": (dataclasses.replace(base, Hq=8, Hkv=2, structure="iid"),
+                         (300, 0, 129), 0.5),
+        "paged_empty": (dataclasses.replace(W["paged"], Hq=8, Hkv=2, structure="iid"),
+                        (0, 200, 0, 65), 0.5),
     }
     w, seqlens, alpha = cases[name]
     return S.make_inputs(w, seed=7, seqlens=seqlens), alpha
@@ -57,7 +62,7 @@ def _case(name):
 
 SMALL = ["tiny", "tiny_a09", "gqa_ragged", "gqa_ragged_a05", "varlen", "paged", "fp8",
          "mha_d128", "dense_alpha0", "d128_b64", "d64_b128", "long_ragged", "varlen_long", "gqa8",
-         "gqa3_ffma"]
+         "gqa3_ffma", "varlen_empty", "paged_empty"]
 # cases whose full fp64 attention would be slow: the oracle runs on every 5th query block
 SAMPLED = {"long_ragged", "varlen_long"}
 
@@ -306,3 +311,30 @@ def _full_size(name, cuda_device, n_rows=48):
 @pytest.mark.parametrize("name", ["llama32k", "llama128k", "fp8_128k", "paged", "chunked"])
 def test_full_size_workloads(name, cuda_device):
     _full_size(name, cuda_device)
+
+
+def test_longest_sequence_512k(cuda_device):
+    """One 524,288-token sequence (4,096 blocks per row): the largest single layer the tests
+    run. Pooled means and the mask against the oracle in full, the attention on sampled rows."""
+    w = dataclasses.replace(W["llama128k"], Hq=8, Hkv=2)
+    inp = S.make_inputs(w, seed=19, seqlens=(524288,))
+    run = OracleRun(inp, w.alpha)
+    q, k, v, _ = device_inputs(inp, cuda_device)
+    b = _batch(inp, cuda_device)
+    qp, kp = fp.pool_qk(q, k, w.block, batch=b)
+    bits, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b)
+    out, _ = fp.sparse_prefill_attn(q, k, v, cnt, idx, w.block, batch=b)
+    fp.check_status(cuda_device)
+    for got, ref in ((qp, run.q_pool), (kp, run.k_pool)):
+        g = got.cpu().double().numpy()
+        assert np.abs(g - ref).max() <= 1e-5 * max(1.0, np.abs(ref).max())
+    gk = bits_to_keeps(bits, run)
+    bad, ex, tot = mask_mismatches(gk, run)
+    assert bad == 0 and ex <= max(4, tot // 100000), (bad, ex, tot)
+    rng = np.random.default_rng(23)
+    rows = [(int(rng.integers(w.Hq)), int(Ig)) for Ig in rng.integers(0, run.qoff[-1], 24)]
+    rows.append((w.Hq - 1, run.qoff[-1] - 1))
+    rows = [(h, Ig) for h, Ig in rows if np.array_equal(gk[0][h, Ig], run.keeps[0][h, Ig])]
+    ref, _ = run.attention(rows=rows)
+    amax, rel = attn_errors(out, ref)
+    assert amax <= TOL["bf16"][0] and rel <= TOL["bf16"][1], (amax, rel)

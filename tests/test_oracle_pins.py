@@ -308,3 +308,25 @@ def test_chunked_scores_and_keeps_match_the_full_prefill_on_whole_blocks():
             if I * block >= P0:                       # whole block inside the chunk
                 assert np.array_equal(sc_c[b][:, i], sc_f[b][:, I])
                 assert np.array_equal(kc[:, i], kf[:, I])
+
+
+def test_empty_request_contributes_nothing():
+    """A request without tokens has no blocks: a batch that holds one gives every other
+    request exactly what the batch without it gives."""
+    rng = np.random.default_rng(41)
+    B, H, d = 16, 2, 8
+    lens_with, lens_without = (40, 0, 23), (40, 23)
+    T = sum(lens_with)
+    q, k, v = (rng.standard_normal((T, H, d)) for _ in range(3))
+    outs = []
+    for lens in (lens_with, lens_without):
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(int)
+        qp = O.pool_blocks(q, B, cu)
+        kp = O.pool_blocks(k, B, cu)
+        sc = O.block_scores(qp, kp, cu, B, 0.3)
+        keeps = [O.block_keep(s, 0.2) for s in sc]
+        if len(lens) == 3:
+            assert sc[1].shape == (H, 0, 0) and keeps[1].shape == (H, 0, 0)
+            assert O.keep_ratio(sc[1]).shape == (H, 0, 0)
+        outs.append(O.masked_causal_attention(q, k, v, keeps, cu, B, 0.3)[0])
+    assert np.array_equal(outs[0], outs[1])
