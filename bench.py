@@ -112,7 +112,6 @@ class Layer:
         self.k_split = torch.empty(fp.k_split_shape(w.Hkv, nkb, w.d), dtype=torch.bfloat16,
                                    device=dev)
         self.stream = torch.cuda.current_stream(dev)
-        self.ev = []
 
     def step(self, events=None):
         w, b, cb = self.w, self.batch, self.cb

@@ -263,18 +263,6 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// ---- register reallocation between warpgroups ------------------------------------------------
-// Executed by all threads of a warpgroup; the counts must add up (per warpgroup x 128 threads)
-// to no more than the block was launched with.
-template <uint32_t N>
-__device__ __forceinline__ void regs_dealloc() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_alloc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // ---- misc -------------------------------------------------------------------------------------------
 // 2^x with the MUFU approximation (PTX ex2.approx.ftz.f32; ex2(-inf) = +0).
 __device__ __forceinline__ float ex2(float x) {
