@@ -114,11 +114,29 @@ def _check(rc):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a contiguous CUDA tensor (None passes NULL). The kernels read plain
+    row-major device memory, so host tensors and strided views are refused here rather than
+    read wrongly on the GPU."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"expected a contiguous tensor, got shape {tuple(t.shape)} with "
+                         f"strides {t.stride()}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _same_dtype(*ts):
+    """Q, K and V (or a cache) must share one storage type: the kernels read them as one."""
+    ts = [t for t in ts if t is not None]
+    if any(t.dtype != ts[0].dtype for t in ts):
+        raise TypeError("Q, K and V must have the same dtype, got "
+                        + ", ".join(str(t.dtype) for t in ts))
 
 
 def _dtype_code(t):
@@ -215,6 +233,7 @@ def pool_qk(q, k, block=128, *, batch: Batch | None = None, q_scale=None, k_scal
     ``build_block_mask(k_split=...)`` then loads instead of converting."""
     T, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
+    _same_dtype(q, kk)
     Hkv = kk.shape[-2]
     b = _batch_for(q, block, batch)
     q_pool = torch.empty((Hq, b.total_blocks, d), dtype=torch.float32, device=q.device)
@@ -266,6 +285,7 @@ def sparse_prefill_attn(q, k, v, kv_cnt, kv_idx, block=128, *, batch: Batch | No
                         scale=None, q_scale=None, k_scale=None, v_scale=None,
                         return_lse=False, out=None, ws=None):
     """Causal attention over the kept KV blocks -> (out bf16 [T,Hq,d], lse [Hq,T] or None)."""
+    _same_dtype(q, k, v)
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     b = _batch_for(q, block, batch)
@@ -287,6 +307,7 @@ def sparse_prefill_attn_paged(q, paged: PagedKV, kv_cnt, kv_idx, batch: Batch, *
                               scale=None, q_scale=None, k_scale=None, v_scale=None,
                               return_lse=False, out=None, ws=None):
     """Same as ``sparse_prefill_attn`` with K/V read through the page table."""
+    _same_dtype(q, paged.k_cache, paged.v_cache)
     T, Hq, d = q.shape
     Hkv = paged.k_cache.shape[2]
     if scale is None:
@@ -341,6 +362,7 @@ def pool_and_mask_noalloc(q, k, alpha=0.1, block=128, *, batch: Batch | None = N
     kv_cnt, kv_idx); the output tensors are allocated here by torch for convenience."""
     T, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
+    _same_dtype(q, kk)
     Hkv = kk.shape[-2]
     b = _batch_for(q, block, batch)
     if scale is None:
@@ -422,6 +444,7 @@ def pool_qk_chunked(q, k, cb: ChunkedBatch, *, q_scale=None, k_scale=None,
     query block holds, k_pool [Hkv, total_kblocks, d] over all keys (cached prefix included)."""
     _, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
+    _same_dtype(q, kk)
     Hkv = kk.shape[-2]
     q_pool = torch.empty((Hq, cb.total_qblocks, d), dtype=torch.float32, device=q.device)
     k_pool = torch.empty((Hkv, cb.total_kblocks, d), dtype=torch.float32, device=q.device)
@@ -464,6 +487,7 @@ def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
     T, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
     vv = paged.v_cache if paged is not None else v
+    _same_dtype(q, kk, vv)
     Hkv = kk.shape[-2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -486,6 +510,7 @@ def append_paged_kv(k_new, v_new, cb: ChunkedBatch, paged: PagedKV, *, ws=None):
     """Writes the chunk's new K and V rows [total_q, Hkv, d] into the paged caches at their
     absolute positions (before the chunked prefill reads them)."""
     T, Hkv, d = k_new.shape
+    _same_dtype(k_new, v_new, paged.k_cache, paged.v_cache)
     ws = workspace(k_new.device) if ws is None else ws
     pt = paged.page_table
     _check(library().fp_append_paged_kv(

@@ -130,3 +130,28 @@ def test_empty_inputs_return_ok_without_launching():
     assert _bad_attn(T=0, tb=0, mb=0) == 0
     assert lib.fp_append_paged_kv(16, 16, 0, 16, 16, 1, 0, 2, 128, 16, 64, 1, 1, 16, 16, 256,
                                   None) == 0
+
+
+def test_host_index_arrays_are_refused_before_launch():
+    """Prefix sums left in host memory would make a kernel fault the GPU; the library
+    refuses them (on a machine without a GPU the pointer cannot even be queried)."""
+    import numpy as np
+    cu = np.array([0, 200, 300], dtype=np.int32)
+    cb = np.array([0, 2, 3], dtype=np.int32)
+    lib = fp.library()
+    rc = lib.fp_pool_qk(16, 16, 0, None, None, cu.ctypes.data, cb.ctypes.data, 2, 300, 3, 8, 2,
+                        128, 128, None, 0, 0, 0, 16, 16, None, None)
+    assert rc == -1
+    assert b"cu_" in lib.fp_last_error_string()
+
+
+def test_binding_refuses_cpu_tensors_views_and_mixed_dtypes():
+    import torch
+    q = torch.zeros((256, 4, 128), dtype=torch.bfloat16)
+    k = torch.zeros((256, 2, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fp._ptr(q)
+    with pytest.raises(TypeError, match="same dtype"):
+        fp._same_dtype(q, k.to(torch.float8_e4m3fn))
+    fp._same_dtype(q, k, None)
+    assert fp._ptr(None) is None

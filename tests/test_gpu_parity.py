@@ -338,3 +338,25 @@ def test_longest_sequence_512k(cuda_device):
     ref, _ = run.attention(rows=rows)
     amax, rel = attn_errors(out, ref)
     assert amax <= TOL["bf16"][0] and rel <= TOL["bf16"][1], (amax, rel)
+
+
+def test_strided_views_and_host_prefix_sums_are_refused(cuda_device):
+    q = torch.zeros((256, 4, 128), dtype=torch.bfloat16, device=cuda_device)
+    k = torch.zeros((256, 2, 128), dtype=torch.bfloat16, device=cuda_device)
+    with pytest.raises(ValueError, match="contiguous"):
+        fp.pool_qk(q[:, :, :64], k[:, :, :64], 128)
+    b = fp.Batch.make((200, 56), 128, cuda_device)
+    host_b = dataclasses.replace(b, cu_seqlens=b.cu_seqlens.cpu().pin_memory().cuda(),
+                                 cu_blocks=b.cu_blocks.cpu())
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fp.pool_qk(q, k, 128, batch=host_b)
+    # at the C ABI: a host array is refused with a message, nothing is launched
+    import numpy as np
+    cu = np.array([0, 200, 256], dtype=np.int32)
+    qp = torch.empty((4, 3, 128), device=cuda_device)
+    kp = torch.empty((2, 3, 128), device=cuda_device)
+    rc = fp.library().fp_pool_qk(fp._ptr(q), fp._ptr(k), 0, None, None, cu.ctypes.data,
+                                 fp._ptr(b.cu_blocks), 2, 256, 3, 4, 2, 128, 128, None, 0, 0,
+                                 0, fp._ptr(qp), fp._ptr(kp), None, fp._stream(q.device))
+    assert rc == -1 and b"host memory" in fp.library().fp_last_error_string()
+    torch.cuda.synchronize()
