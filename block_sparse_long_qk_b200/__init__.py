@@ -30,7 +30,7 @@ import torch
 
 __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_attn",
            "sparse_prefill_attn_paged", "sparse_prefill", "check_status", "workspace",
-           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "header_symbols",
+           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "MASK_FP32", "header_symbols",
            "pool_and_mask_noalloc", "k_split_shape", "ChunkedBatch", "pool_qk_chunked",
            "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked",
            "HostPipeline", "append_paged_kv"]
@@ -41,7 +41,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "fpsparse.h")
 
 FP_OK = 0
 FP_DTYPE_BF16, FP_DTYPE_E4M3 = 0, 1
-FORCE_FIRST, FORCE_DIAG = 1, 2
+FORCE_FIRST, FORCE_DIAG, MASK_FP32 = 1, 2, 4
 _ERRORS = {-1: "FP_ERR_INVALID_ARG", -2: "FP_ERR_UNSUPPORTED", -3: "FP_ERR_CUDA",
            -4: "FP_ERR_TIMEOUT", -5: "FP_ERR_BAD_INDEX"}
 

@@ -212,9 +212,10 @@ int mask_impl(const float* q_pool, const float* k_pool, const void* k_pool_split
   if (rc) return rc;
   const int G = Hq / Hkv;
   const int nb = fp::mask_blocks_per_cta(G, d, s.max_kb);
-  if (nb == 0 && !fp::mask_tc_supported(G, d))
+  const bool fp32 = (flags & FP_MASK_FP32) != 0 || !fp::mask_tc_supported(G, d);
+  if (fp32 && nb == 0)
     return fail(FP_ERR_UNSUPPORTED, "%d blocks per request with %d heads per KV head exceed the "
-                "shared-memory score rows of the mask kernel", s.max_kb, G);
+                "shared-memory score rows of the fp32 mask kernel", s.max_kb, G);
   fp::MaskArgs a{};
   a.q_pool = q_pool;
   a.k_pool = k_pool;
@@ -269,8 +270,8 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
   a.page_size = page_size;
   a.max_pages = max_pages;
   a.num_pages = num_pages;
-  a.pair_heads = (G % 2 == 0) ? 1 : 0;
-  a.num_items = a.pair_heads ? (Hq / 2) * s.total_qb : Hq * s.total_qb;
+  a.G = G;
+  a.num_items = Hkv * ((G + 1) / 2) * s.total_qb;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.fault_skip_k = g_fault_skip_k;
   g_fault_skip_k = -1;

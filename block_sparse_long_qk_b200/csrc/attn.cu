@@ -110,24 +110,21 @@ struct UnionWalk {
 // position 0 and its key count; `b`: the request (page-table row).
 __device__ __forceinline__ void make_tiles(const AttnArgs& a, int item, Tile* t, int& g,
                                            int& b, int& kbase, int& len) {
-  int Ig;
-  if (a.pair_heads) {
-    const int npairs = a.Hq / 2;
-    Ig = a.s.total_qb - 1 - item / npairs;
-    const int p = item % npairs;
-    for (int s = 0; s < 2; ++s) { t[s].h = 2 * p + s; t[s].Ig = Ig; }
-  } else {
-    // Query heads do not pair up on a KV head (odd group size): one tile per CTA.
-    Ig = a.s.total_qb - 1 - item / a.Hq;
-    const int h = item % a.Hq;
-    t[0].h = h; t[0].Ig = Ig;
-    t[1].h = h; t[1].Ig = -1;
-  }
+  // The G query heads of a KV head form ceil(G / 2) items per query block: pairs of heads, and
+  // for an odd G one single head (its CTA runs one tile).
+  const int npair = (a.G + 1) / 2;
+  const int per_block = a.Hkv * npair;
+  const int Ig = a.s.total_qb - 1 - item / per_block;
+  const int rem = item % per_block;
+  g = rem / npair;
+  const int h0 = g * a.G + 2 * (rem % npair);
+  t[0].h = h0; t[0].Ig = Ig;
+  t[1].h = h0 + 1; t[1].Ig = (h0 + 1 < (g + 1) * a.G) ? Ig : -1;
+  if (t[1].Ig < 0) t[1].h = h0;
   const QBlock qb = query_block(a.s, Ig);
   b = qb.b;
   kbase = qb.kbase;
   len = qb.L;
-  g = t[0].h / (a.Hq / a.Hkv);
   for (int s = 0; s < 2; ++s) {
     if (t[s].Ig < 0) {
       t[s].r0 = t[s].r1 = 0; t[s].cnt = 0; t[s].list = a.kv_idx; t[s].I = -1; t[s].q_lo = 0;

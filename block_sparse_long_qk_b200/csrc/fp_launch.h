@@ -64,8 +64,8 @@ struct AttnArgs {
   Seqs s;
   int Hq, Hkv;
   int page_size, max_pages, num_pages;  // paged only
-  int pair_heads;                       // 1: the two tiles of a CTA are two heads of one block
-  int num_items;
+  int G;                               // query heads per KV head
+  int num_items;                        // Hkv * ceil(G / 2) * total_qb
   int fault_skip_k;                     // test hook: CTA 0 skips the K load of this union block
   float scale_log2;                     // softmax scale * log2(e)
 };

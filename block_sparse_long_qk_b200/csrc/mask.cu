@@ -7,6 +7,9 @@
 // s_J - max s >= ln(alpha) on the scaled pooled logits, which is what runs here (the softmax
 // denominator cancels, so no exponential is needed).
 //
+// Used when the caller asks for fp32 scores (FP_MASK_FP32), as an independent implementation of
+// the same stage next to the tensor-core kernel in mask_tc.cu.
+//
 // One CTA owns R = G * NB rows: the G query heads that share KV head g, times NB consecutive
 // global query blocks. It streams the KV head's pooled keys through shared memory in chunks
 // of 64 blocks, so every pooled key row is read from L2 once per CTA and reused by all R rows,
@@ -177,7 +180,8 @@ int mask_blocks_per_cta(int G, int d, int max_blocks) {
 }
 
 cudaError_t launch_mask(const MaskArgs& in, cudaStream_t stream) {
-  if (mask_tc_supported(in.G, in.d)) return launch_mask_tc(in, stream);
+  if (!(in.flags & FP_MASK_FP32) && mask_tc_supported(in.G, in.d))
+    return launch_mask_tc(in, stream);
   MaskArgs a = in;
   const size_t smem = mask_smem_bytes(a.G * a.NB, a.d, a.s.max_kb);
   cudaError_t e = cudaFuncSetAttribute(mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

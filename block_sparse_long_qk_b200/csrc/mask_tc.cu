@@ -10,8 +10,9 @@
 // which leaves a relative error of about 3 * 2^-18 of sum |q_c k_c| (the dropped q_lo . k_lo and
 // the bf16 rounding of the residuals).
 //
-// One CTA = 128 query rows (the G heads of KV head g times 128/G consecutive query blocks) x
-// every key block its rows need, in chunks of 128 key blocks: S = Q K^T is an M=128, N=128,
+// One CTA = 128 query rows (the G heads of KV head g times floor(128/G) consecutive query
+// blocks; when G does not divide 128 the last 128 mod G rows stay empty) x every key block its
+// rows need, in chunks of 128 key blocks: S = Q K^T is an M=128, N=128,
 // K=d tile. Pass 0 takes each row's max over its causal, same-request blocks; pass 1 recomputes
 // the chunks and writes the keep bits and the ascending index list. Operands are converted
 // from fp32 and written to shared memory in the 128-byte-swizzled K-major layout by all 512
@@ -94,13 +95,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // the longest causal rows -- launch first and the short ones fill the tail.
   const int g = blockIdx.x % a.Hkv;
   const int rows_blk = kTcRows / a.G;                 // query blocks per CTA
+  const int rows_used = rows_blk * a.G;               // the rest (when G does not divide 128) idle
   const int ntiles = gridDim.x / a.Hkv;
   const int Ig0 = (ntiles - 1 - static_cast<int>(blockIdx.x) / a.Hkv) * rows_blk;
 
   if (tid < kTcRows) {
     const int Ig = Ig0 + tid / a.G;
     row_h[tid] = g * a.G + tid % a.G;
-    if (Ig < a.s.total_qb) {
+    if (tid < rows_used && Ig < a.s.total_qb) {
       const QBlock qb = query_block(a.s, Ig);
       row_I[tid] = qb.I;     // absolute query block: keys J = 0 .. I of the request
       row_kb[tid] = qb.kb0;  // global KV block of the request's block 0
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int i = tid; i < kTcRows * words; i += kTcThreads) {
       const int rr = i / words;
       const int Ig = Ig0 + rr / a.G;
-      if (Ig < a.s.total_qb)
+      if (rr < rows_used && Ig < a.s.total_qb)
         a.mask_bits[(static_cast<size_t>(g * a.G + rr % a.G) * a.s.total_qb + Ig) * words +
                     i % words] = 0u;
     }
@@ -141,7 +143,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int r = u / kUnits, k0 = (u % kUnits) * 8;
     const int Ig = Ig0 + r / a.G;
     float v[8];
-    if (Ig < a.s.total_qb) {
+    if (r < rows_used && Ig < a.s.total_qb) {
       const float4* src = reinterpret_cast<const float4*>(
           a.q_pool + (static_cast<size_t>(g * a.G + r % a.G) * a.s.total_qb + Ig) * D + k0);
       const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }  // namespace
 
 bool mask_tc_supported(int G, int d) {
-  return (d == 64 || d == 128) && G >= 1 && G <= kTcRows && kTcRows % G == 0;
+  return (d == 64 || d == 128) && G >= 1 && G <= kTcRows;
 }
 
 template <int D, bool kTma>

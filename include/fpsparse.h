@@ -60,6 +60,8 @@ extern "C" {
 
 #define FP_FORCE_FIRST 1 /* always keep KV block 0 of every row */
 #define FP_FORCE_DIAG 2  /* always keep the diagonal KV block J = I */
+#define FP_MASK_FP32 4   /* pooled scores in fp32 FFMA instead of the tensor cores (slower; the
+                            same keep rule, a second implementation to cross-check) */
 
 /* Library version, e.g. 100 for 0.1.0. */
 int fp_version(void);
@@ -103,6 +105,9 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
  *   s_J  = scale * dot(q_pool[h, Ig], k_pool[h / (Hq/Hkv), cu_blocks[b] + J])   (float32)
  *   keep J  iff  s_J - max_J s_J >= ln(alpha)          (= softmax(s)_J >= alpha * max softmax)
  *           or (flags & FP_FORCE_FIRST and J == 0) or (flags & FP_FORCE_DIAG and J == I).
+ * flags may also hold FP_MASK_FP32 (fp32 FFMA scores instead of the tensor cores; that kernel
+ * keeps a request's score rows in shared memory, so very long requests with it return
+ * FP_ERR_UNSUPPORTED).
  * alpha in [0, 1]; alpha = 0 keeps every causal block.
  *
  * k_pool_split  NULL, or the split written by fp_pool_qk for this k_pool (results are

@@ -34,7 +34,8 @@ CASES = {
     "paged": (dataclasses.replace(BASE, page_size=64), (1000, 700, 300), (333, 700, 65), 0.5),
     "fp8": (dataclasses.replace(BASE, dtype="e4m3"), (1100, 600), (450, 130), 0.5),
     "b64_d64": (dataclasses.replace(BASE, block=64, d=64), (700, 333), (250, 90), 0.5),
-    "gqa3_ffma": (dataclasses.replace(BASE, Hq=6), (800, 500), (300, 77), 0.5),
+    "gqa3": (dataclasses.replace(BASE, Hq=6), (800, 500), (300, 77), 0.5),
+    "gqa5": (dataclasses.replace(BASE, Hq=10, structure="band"), (900, 1300), (450, 129), 0.1),
     # many key blocks per row (several score chunks in the mask kernel), long cached prefix
     "long_prefix": (dataclasses.replace(W["llama128k"], Hq=8, Hkv=2), (20000, 9000),
                     (1500, 2700), 0.1),

@@ -48,8 +48,11 @@ def _case(name):
                         (17000, 300, 9000), 0.5),
         # group of 8 query heads per KV head
         "gqa8": (dataclasses.replace(base, Hq=16, Hkv=2, structure="iid"), (3000,), 0.5),
-        # group of 3: the fp32 FFMA mask kernel and single-tile attention CTAs
-        "gqa3_ffma": (dataclasses.replace(base, Hq=6, Hkv=2, structure="iid"), (1500,), 0.5),
+        # groups of 3, 5 and 7: mask row tiles with idle rows (G does not divide 128), and
+        # attention CTAs holding a pair of heads or a single one
+        "gqa3": (dataclasses.replace(base, Hq=6, Hkv=2, structure="iid"), (1500,), 0.5),
+        "gqa5": (dataclasses.replace(base, Hq=10, Hkv=2, structure="band"), (1300, 700), 0.1),
+        "gqa7": (dataclasses.replace(base, Hq=7, Hkv=1, structure="band"), (1500,), 0.1),
         # a request without tokens between two others (no blocks, no rows)
         "varlen_empty": (dataclasses.replace(base, Hq=8, Hkv=2, structure="iid"),
                          (300, 0, 129), 0.5),
@@ -62,7 +65,7 @@ def _case(name):
 
 SMALL = ["tiny", "tiny_a09", "gqa_ragged", "gqa_ragged_a05", "varlen", "paged", "fp8",
          "mha_d128", "dense_alpha0", "d128_b64", "d64_b128", "long_ragged", "varlen_long", "gqa8",
-         "gqa3_ffma", "varlen_empty", "paged_empty"]
+         "gqa3", "gqa5", "gqa7", "varlen_empty", "paged_empty"]
 # cases whose full fp64 attention would be slow: the oracle runs on every 5th query block
 SAMPLED = {"long_ragged", "varlen_long"}
 
@@ -360,3 +363,30 @@ def test_strided_views_and_host_prefix_sums_are_refused(cuda_device):
                                  0, fp._ptr(qp), fp._ptr(kp), None, fp._stream(q.device))
     assert rc == -1 and b"host memory" in fp.library().fp_last_error_string()
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("name", ["tiny", "gqa3", "varlen", "gqa8"])
+def test_fp32_mask_matches_oracle_and_tensor_core_mask(name, cuda_device):
+    """FP_MASK_FP32 runs the fp32 FFMA scores: the same keep sets as the oracle (up to the
+    near-threshold exemption), and as the tensor-core kernel away from the threshold."""
+    inp, alpha = _case(name)
+    run = OracleRun(inp, alpha)
+    q, k, _, sc = device_inputs(inp, cuda_device)
+    b = _batch(inp, cuda_device)
+    qp, kp = fp.pool_qk(q, k, inp.workload.block, batch=b, q_scale=sc["q_scale"],
+                        k_scale=sc["k_scale"], paged=_paged(inp, cuda_device))
+    flags = fp.FORCE_FIRST | fp.FORCE_DIAG
+    bits32, cnt32, idx32 = fp.build_block_mask(qp, kp, alpha, block=inp.workload.block, batch=b,
+                                               flags=flags | fp.MASK_FP32)
+    bits, _, _ = fp.build_block_mask(qp, kp, alpha, block=inp.workload.block, batch=b,
+                                     flags=flags)
+    torch.cuda.synchronize()
+    g32 = bits_to_keeps(bits32, run)
+    bad, ex, tot = mask_mismatches(g32, run)
+    assert bad == 0 and ex <= max(2, tot // 1000), (bad, ex, tot)
+    for a_, b_ in zip(g32, lists_to_keeps(cnt32, idx32, run)):
+        assert np.array_equal(a_, b_)
+    gtc = bits_to_keeps(bits, run)
+    for r, (x, y, ratio) in enumerate(zip(g32, gtc, run.ratios)):
+        near = np.abs(ratio - alpha) <= 1e-3 * alpha
+        assert not ((x != y) & ~near).any()
