@@ -33,7 +33,7 @@ __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_at
            "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "MASK_FP32", "header_symbols",
            "pool_and_mask_noalloc", "k_split_shape", "ChunkedBatch", "pool_qk_chunked",
            "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked",
-           "HostPipeline", "append_paged_kv"]
+           "HostPipeline", "append_paged_kv", "GraphStep"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfpsparse.so")
@@ -592,3 +592,29 @@ class HostPipeline:
     def synchronize(self):
         for st in (self.h2d, self.comp, self.d2h):
             st.synchronize()
+
+
+class GraphStep:
+    """One step of the path captured into a CUDA graph: ``run(*inputs)`` (device tensors of
+    fixed shape, the call's other arguments bound) is run ``warmup`` times eagerly, then
+    captured; ``replay()`` relaunches all of its kernels at once and returns the tensors the
+    captured call returned. New data goes into the captured input tensors in place
+    (``inputs[i].copy_(...)``) before a replay. The library's calls allocate nothing on the
+    device and never synchronise, so they capture as they are."""
+
+    def __init__(self, run, inputs, warmup=2):
+        self.inputs = tuple(inputs)
+        dev = self.inputs[0].device
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                run(*self.inputs)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.outputs = run(*self.inputs)
+
+    def replay(self):
+        self.graph.replay()
+        return self.outputs

@@ -34,8 +34,16 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // The small index arrays (prefix sums, page tables) are the arguments most easily left in
 // host memory by a caller; a kernel reading one would fault the GPU. Each non-NULL one must
-// be memory the device can address.
-int check_device_arrays(std::initializer_list<std::pair<const void*, const char*>> arrays) {
+// be memory the device can address. While `stream` is being captured into a CUDA graph the
+// query is skipped (it is not a stream operation; the same call run eagerly checks it).
+int check_device_arrays(void* stream,
+                        std::initializer_list<std::pair<const void*, const char*>> arrays) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cs) != cudaSuccess) {
+    cudaGetLastError();
+    cs = cudaStreamCaptureStatusNone;
+  }
+  if (cs != cudaStreamCaptureStatusNone) return FP_OK;
   for (const auto& a : arrays) {
     if (a.first == nullptr) continue;
     cudaPointerAttributes at{};
@@ -172,9 +180,9 @@ int pool_impl(const void* q, const void* k, int dtype, const float* q_scale,
   if (k_page_table && s.cu_k == nullptr)
     return fail(FP_ERR_INVALID_ARG, "a paged K needs the varlen prefix sums");
   if (s.total_kb == 0) return FP_OK;
-  rc = check_device_arrays({{s.cu_q, "cu_q / cu_seqlens"}, {s.cu_qb, "cu_qblocks / cu_blocks"},
-                            {s.cu_k, "cu_k"}, {s.cu_kb, "cu_kblocks"},
-                            {k_page_table, "k_page_table"}});
+  rc = check_device_arrays(stream, {{s.cu_q, "cu_q / cu_seqlens"},
+                                    {s.cu_qb, "cu_qblocks / cu_blocks"}, {s.cu_k, "cu_k"},
+                                    {s.cu_kb, "cu_kblocks"}, {k_page_table, "k_page_table"}});
   if (rc) return rc;
   fp::PoolArgs a{};
   a.q = static_cast<const uint8_t*>(q);
@@ -207,8 +215,8 @@ int mask_impl(const float* q_pool, const float* k_pool, const void* k_pool_split
   if (!aligned16(q_pool) || !aligned16(k_pool) || !aligned16(k_pool_split))
     return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
   if (s.total_qb == 0) return FP_OK;
-  int rc = check_device_arrays({{s.cu_q, "cu_q"}, {s.cu_qb, "cu_qblocks / cu_blocks"},
-                                {s.cu_k, "cu_k"}, {s.cu_kb, "cu_kblocks"}});
+  int rc = check_device_arrays(stream, {{s.cu_q, "cu_q"}, {s.cu_qb, "cu_qblocks / cu_blocks"},
+                                        {s.cu_k, "cu_k"}, {s.cu_kb, "cu_kblocks"}});
   if (rc) return rc;
   const int G = Hq / Hkv;
   const int nb = fp::mask_blocks_per_cta(G, d, s.max_kb);
@@ -285,10 +293,11 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
   L.kv_rows = page_table ? static_cast<long long>(num_pages) * page_size : s.total_k;
   L.seg_rows = page_table ? page_size : s.block;
   if (s.total_qb == 0) return FP_OK;
-  rc = check_device_arrays({{s.cu_q, "cu_q / cu_seqlens"}, {s.cu_qb, "cu_qblocks / cu_blocks"},
-                            {s.cu_k, "cu_k"}, {s.cu_kb, "cu_kblocks"},
-                            {page_table, "page_table"}, {kv_cnt, "kv_cnt"}, {kv_idx, "kv_idx"},
-                            {workspace, "workspace"}});
+  rc = check_device_arrays(stream, {{s.cu_q, "cu_q / cu_seqlens"},
+                                    {s.cu_qb, "cu_qblocks / cu_blocks"}, {s.cu_k, "cu_k"},
+                                    {s.cu_kb, "cu_kblocks"}, {page_table, "page_table"},
+                                    {kv_cnt, "kv_cnt"}, {kv_idx, "kv_idx"},
+                                    {workspace, "workspace"}});
   if (rc) return rc;
   cudaError_t e = fp::launch_attn(a, L, s.block, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return fail(FP_ERR_UNSUPPORTED, "unsupported d/block/dtype");
@@ -481,8 +490,8 @@ int fp_append_paged_kv(const void* k_new, const void* v_new, int dtype, const in
   if (page_size < 1 || max_pages < 1 || num_pages < 1)
     return fail(FP_ERR_INVALID_ARG, "page_size, max_pages and num_pages must be >= 1");
   if (total_q == 0) return FP_OK;
-  int rc = check_device_arrays({{cu_q, "cu_q"}, {cu_k, "cu_k"}, {page_table, "page_table"},
-                                {workspace, "workspace"}});
+  int rc = check_device_arrays(stream, {{cu_q, "cu_q"}, {cu_k, "cu_k"},
+                                        {page_table, "page_table"}, {workspace, "workspace"}});
   if (rc) return rc;
   fp::AppendArgs a{};
   a.k_new = static_cast<const uint8_t*>(k_new);
