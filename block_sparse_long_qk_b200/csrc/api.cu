@@ -116,7 +116,7 @@ int set_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int fp_version(void) { return 100; }
+int fp_version(void) { return 110; }
 
 const char* fp_last_error_string(void) { return g_err.c_str(); }
 

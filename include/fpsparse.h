@@ -63,7 +63,8 @@ extern "C" {
 #define FP_MASK_FP32 4   /* pooled scores in fp32 FFMA instead of the tensor cores (slower; the
                             same keep rule, a second implementation to cross-check) */
 
-/* Library version, e.g. 100 for 0.1.0. */
+/* Library version, e.g. 110 for 0.1.1 (0.1.1 adds the chunked-prefill calls, the paged K/V
+ * append and FP_MASK_FP32). */
 int fp_version(void);
 
 /* Message describing the last error returned on the calling thread ("" if none). */
