@@ -2,18 +2,20 @@
 // the paged KV cache at their absolute positions ("FlashPrefill V2: Block-Sparse Prefill
 // Attention for Long-Context LLM Serving", Abstract: paged KV cache and continuous batching).
 //
-// Pure data movement: one CTA per new token row, each thread moving 16-byte units of the
-// row's Hkv x d elements from the contiguous chunk to (page, slot) of the cache, K and V.
+// Pure data movement: one CTA per 8 new token rows, each thread moving 16-byte units of the
+// rows' Hkv x d elements from the contiguous chunk to (page, slot) of the cache, K and V, with
+// the 8 rows' loads in flight together.
 #include "fp_common.cuh"
 #include "fp_launch.h"
 
 namespace fp {
 
 constexpr int kAppendThreads = 128;
+constexpr int kAppendRows = 8;  // new rows per CTA, their loads in flight together
 
-__global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
-  const int t = blockIdx.x;  // new row
-  if (t >= a.s.total_q) return;
+// Destination row of new row t in the cache, or -1 (and the status bit) when its page entry is
+// out of range.
+__device__ __forceinline__ long long append_dst_row(const AppendArgs& a, int t) {
   const int b = seqs_find(a.s.cu_q, a.s.batch, t);
   const int q0 = __ldg(a.s.cu_q + b);
   const int n = __ldg(a.s.cu_q + b + 1) - q0;
@@ -21,27 +23,51 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
   const int p = L - n + (t - q0);  // absolute position of the row
   const int lp = p / a.page_size;
   int page = -1;
-  if (p >= 0 && lp < a.max_pages) page = __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp);
-  if (page < 0 || page >= a.num_pages) {
-    if (threadIdx.x == 0) record_status(a.status, kStatusBadIndex);
-    return;
-  }
-  const size_t dst_row = static_cast<size_t>(page) * a.page_size + p % a.page_size;
+  if (p >= 0 && lp < a.max_pages)
+    page = __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp);
+  if (page < 0 || page >= a.num_pages) return -1;
+  return static_cast<long long>(page) * a.page_size + p % a.page_size;
+}
+
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendArgs a) {
+  const int t0 = blockIdx.x * kAppendRows;
   const int units = a.row_bytes / 16;
-  const int4* ks = reinterpret_cast<const int4*>(a.k_new + static_cast<size_t>(t) * a.row_bytes);
-  const int4* vs = reinterpret_cast<const int4*>(a.v_new + static_cast<size_t>(t) * a.row_bytes);
-  int4* kd = reinterpret_cast<int4*>(a.k_cache + dst_row * a.row_bytes);
-  int4* vd = reinterpret_cast<int4*>(a.v_cache + dst_row * a.row_bytes);
+  __shared__ long long dst[kAppendRows];
+  if (threadIdx.x < kAppendRows) {
+    const int t = t0 + threadIdx.x;
+    long long d = -2;  // past the end of the chunk: nothing to do
+    if (t < a.s.total_q) {
+      d = append_dst_row(a, t);
+      if (d < 0) record_status(a.status, kStatusBadIndex);
+    }
+    dst[threadIdx.x] = d;
+  }
+  __syncthreads();
   for (int u = threadIdx.x; u < units; u += blockDim.x) {
-    const int4 kv = __ldcs(ks + u), vv = __ldcs(vs + u);
-    kd[u] = kv;
-    vd[u] = vv;
+    int4 kv[kAppendRows], vv[kAppendRows];
+#pragma unroll
+    for (int r = 0; r < kAppendRows; ++r) {
+      if (dst[r] >= 0) {
+        const size_t src = (static_cast<size_t>(t0 + r) * a.row_bytes) / 16 + u;
+        kv[r] = __ldcs(reinterpret_cast<const int4*>(a.k_new) + src);
+        vv[r] = __ldcs(reinterpret_cast<const int4*>(a.v_new) + src);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kAppendRows; ++r) {
+      if (dst[r] >= 0) {
+        const size_t o = (static_cast<size_t>(dst[r]) * a.row_bytes) / 16 + u;
+        reinterpret_cast<int4*>(a.k_cache)[o] = kv[r];
+        reinterpret_cast<int4*>(a.v_cache)[o] = vv[r];
+      }
+    }
   }
 }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   if (a.s.total_q == 0) return cudaSuccess;
-  append_kernel<<<a.s.total_q, kAppendThreads, 0, stream>>>(a);
+  const int grid = (a.s.total_q + kAppendRows - 1) / kAppendRows;
+  append_kernel<<<grid, kAppendThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
