@@ -1,0 +1,42 @@
+"""Host-side accounting of bench.py: query blocks, work counts and bytes agree with the
+definitions the oracle uses (no GPU)."""
+import numpy as np
+import torch
+
+import oracle as O
+from block_sparse_long_qk_b200 import synthetic as S
+
+import bench
+
+
+def test_query_blocks_match_the_oracle():
+    for name in ("llama128k", "paged", "chunked"):
+        w = S.WORKLOADS[name]
+        cu_k = np.concatenate([[0], np.cumsum(w.seqlens)]).astype(int)
+        q_lens = w.q_lens if w.q_lens is not None else w.seqlens
+        cu_q = np.concatenate([[0], np.cumsum(q_lens)]).astype(int)
+        info, off = O.query_blocks(cu_q, cu_k if w.q_lens is not None else None, w.block)
+        I, lo, hi = bench._query_blocks(w)
+        assert len(I) == off[-1]
+        exp_I = [i0 + i for (_, i0, nq) in info for i in range(nq)]
+        assert I.tolist() == exp_I
+        assert int((hi - lo).sum()) == int(sum(q_lens))
+
+
+def test_work_counts_dense_closed_form():
+    """With every causal block kept, the algorithmic FLOPs are 4 d times the number of causal
+    (query, key) pairs, L (L + 1) / 2 per head for one sequence."""
+    w = S.Workload("t", (1000,), 4, 2, 64, 128)
+    nq = (1000 + 127) // 128
+    cnt = torch.tensor([[I + 1 for I in range(nq)]] * w.Hq, dtype=torch.int32)
+    alg, executed, density = bench.work_counts(w, cnt, None)
+    assert alg == 4.0 * w.d * w.Hq * (1000 * 1001 // 2)
+    assert executed == 4.0 * 128 * 128 * w.d * float(cnt.sum())
+    assert density == 1.0
+
+
+def test_pool_mask_bytes():
+    w = S.WORKLOADS["llama128k"]
+    pool, total = bench.pool_mask_bytes(w)
+    assert pool == 131072 * (32 + 8) * 128 * 2 + (1024 * 32 + 1024 * 8) * 128 * 4 + 1024 * 8 * 128 * 4
+    assert total - pool == (1024 * 32 + 1024 * 8) * 128 * 4 + 1024 * 8 * 128 * 4
