@@ -346,17 +346,21 @@ __global__ void __launch_bounds__(384, 1)
     // with 1/2, 8.76 with none). With bf16 the extra FMA work costs more than it saves, so
     // every exponential uses MUFU ex2.
     constexpr bool kPolyExp = FP8;
-    auto p_pass = [&](float mu, auto diag_tag) -> float {
+    auto p_pass = [&](const float* s_lo, float mu, auto diag_tag) -> float {
       constexpr bool diag = decltype(diag_tag)::value;
       const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-mu, -mu);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
 #pragma unroll
       for (int h0 = 0; h0 < BN; h0 += 64) {
-        float sv[64];
-        tmem_ld32(s_tm + h0, sv);
-        if constexpr (BN > 32) tmem_ld32(s_tm + h0 + 32, sv + 32);
-        tmem_ld_wait();
+        // Columns 0..63 are still in registers from the max pass; the rest is re-read.
+        float sv_hi[64];
+        if (h0 > 0) {
+          tmem_ld32(s_tm + h0, sv_hi);
+          tmem_ld32(s_tm + h0 + 32, sv_hi + 32);
+          tmem_ld_wait();
+        }
+        const float* sv = h0 == 0 ? s_lo : sv_hi;
 #pragma unroll
         for (int c1 = 0; c1 < 64 && h0 + c1 < BN; c1 += 32) {
           const int c0 = h0 + c1;
@@ -405,18 +409,16 @@ __global__ void __launch_bounds__(384, 1)
       float mr[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mr[e] = -INFINITY;
-      {
-        float sv[BN];
+      float sv[BN];
 #pragma unroll
-        for (int c = 0; c < BN; c += 32) tmem_ld32(s_tm + c, sv + c);
-        tmem_ld_wait();
-        if (diag) {
+      for (int c = 0; c < BN; c += 32) tmem_ld32(s_tm + c, sv + c);
+      tmem_ld_wait();
+      if (diag) {
 #pragma unroll
-          for (int c = 0; c < BN; ++c) sv[c] = (c > r) ? -INFINITY : sv[c];
-        }
-#pragma unroll
-        for (int c = 0; c < BN; c += 2) mr[(c / 2) % 8] = fmax3(mr[(c / 2) % 8], sv[c], sv[c + 1]);
+        for (int c = 0; c < BN; ++c) sv[c] = (c > r) ? -INFINITY : sv[c];
       }
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) mr[(c / 2) % 8] = fmax3(mr[(c / 2) % 8], sv[c], sv[c + 1]);
       const float mx = fmax3(fmax3(mr[0], mr[1], mr[2]), fmax3(mr[3], mr[4], mr[5]),
                              fmaxf(mr[6], mr[7])) * sl2;  // sl2 > 0: max commutes with scaling
       // Lazy rescaling: keep the stale max m unless the row max grew by more than 2^8, so P
@@ -432,7 +434,7 @@ __global__ void __launch_bounds__(384, 1)
         rescale = true;
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
-      const float sum = diag ? p_pass(mu, std::true_type{}) : p_pass(mu, std::false_type{});
+      const float sum = diag ? p_pass(sv, mu, std::true_type{}) : p_pass(sv, mu, std::false_type{});
       l += sum;
       // tcgen05.ld/st are warp-collective: when any row of the warp rescales, the whole warp
       // runs the pass (f = 1 for rows that keep their max).
