@@ -337,30 +337,25 @@ __global__ void __launch_bounds__(384, 1)
     int n = 0;
     bool ok = true;
     int i = 0;
-    // P = 2^(s * sl2 - mu) for the row, re-read from TMEM 64 columns at a time (so the whole
-    // S row never has to stay in registers), packed and written over the S columns already
-    // read; returns the row sum. Four independent partial sums keep the add chain short.
+    // P = 2^(s * sl2 - mu) for the row, taken from the S row the max pass left in registers
+    // (no second TMEM read: measured 0.8 % fewer cycles per union block than re-reading the
+    // upper 64 columns, about 3.5 % fewer than re-reading the whole row), packed and written
+    // over the S columns in TMEM; returns the row sum. Four independent partial sums keep the
+    // add chain short.
     // With e4m3 inputs the MMAs run twice as fast and the MUFU ex2 unit (4 lanes per clock per
     // SM sub-partition) becomes the limit: there, three column pairs in eight off the diagonal
     // take the FMA-pipe polynomial instead (measured at 128K: 8.10 ms vs 8.27 with 1/4, 8.57
     // with 1/2, 8.76 with none). With bf16 the extra FMA work costs more than it saves, so
     // every exponential uses MUFU ex2.
     constexpr bool kPolyExp = FP8;
-    auto p_pass = [&](const float* s_lo, float mu, auto diag_tag) -> float {
+    auto p_pass = [&](const float* s_row, float mu, auto diag_tag) -> float {
       constexpr bool diag = decltype(diag_tag)::value;
       const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-mu, -mu);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
 #pragma unroll
       for (int h0 = 0; h0 < BN; h0 += 64) {
-        // Columns 0..63 are still in registers from the max pass; the rest is re-read.
-        float sv_hi[64];
-        if (h0 > 0) {
-          tmem_ld32(s_tm + h0, sv_hi);
-          tmem_ld32(s_tm + h0 + 32, sv_hi + 32);
-          tmem_ld_wait();
-        }
-        const float* sv = h0 == 0 ? s_lo : sv_hi;
+        const float* sv = s_row + h0;
 #pragma unroll
         for (int c1 = 0; c1 < 64 && h0 + c1 < BN; c1 += 32) {
           const int c0 = h0 + c1;
