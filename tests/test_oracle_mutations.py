@@ -42,6 +42,24 @@ MUTANTS = [
      P.test_chunked_query_pool_closed_form),                                  # prefix in the mean
     ("query_blocks", "I0 = P0 // block", "I0 = (P0 + block - 1) // block",
      P.test_chunked_alpha0_equals_dense_rows_of_the_full_sequence),           # first block lost
+    ("query_blocks", "nq = (L + block - 1) // block - I0 if n > 0 else 0",
+     "nq = (L + block - 1) // block - I0",
+     P.test_chunked_request_without_new_queries_has_no_query_block),         # block of no query
+    ("block_scores", "kb = k_pool[h // G, koff[b]:koff[b] + n]",
+     "kb = k_pool[h % Hkv, koff[b]:koff[b] + n]",
+     P.test_pooled_score_is_mean_of_raw_block_scores),                        # wrong KV head
+    ("masked_causal_attention", "k_scale[h // G]", "k_scale[h % Hkv]",
+     P.test_per_head_scale_equals_prescaled_values),                          # wrong K scale
+    ("masked_causal_attention", "(m + np.log(z))", "(np.log(z))",
+     P.test_alpha0_keeps_every_causal_block_and_equals_dense_bruteforce),   # LSE without max
+    ("_row_softmax", "e = np.exp(s - m)", "e = np.exp(s)",
+     lambda: P.test_row_max_always_kept_and_alpha_limits(0.1)),               # overflowing softmax
+    ("block_keep", "keep &= causal[None]", "pass",
+     P.test_alpha0_keeps_every_causal_block_and_equals_dense_bruteforce),   # blocks past diagonal
+    ("pool_blocks", "hi = min(cu[b + 1], lo + block)", "hi = lo + block",
+     P.test_partial_last_block_mean_closed_form),                             # tail past request
+    ("request_blocks", "(cu[b + 1] - cu[b] + block - 1) // block", "(cu[b + 1] - cu[b]) // block",
+     P.test_partial_last_block_mean_closed_form),                             # ragged block lost
 ]
 
 

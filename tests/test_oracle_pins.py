@@ -76,9 +76,11 @@ def test_alpha0_keeps_every_causal_block_and_equals_dense_bruteforce():
 def test_pooled_score_is_mean_of_raw_block_scores():
     """Linearity behind the fused 2-D reduction: qbar_I . kbar_J * scale equals the mean
     over the (valid) I x J rectangle of the raw scaled scores q_i . k_j. Above the block
-    diagonal the pooled row is masked (-inf)."""
+    diagonal the pooled row is masked (-inf). Three query heads per KV head, so that a wrong
+    head mapping (h % Hkv instead of h // G) changes the scores."""
     cu = [0, 40, 40 + 29]
-    Hq, Hkv, d, block = 2, 1, 4, 8
+    Hq, Hkv, d, block = 6, 2, 4, 8
+    G = Hq // Hkv
     T = cu[-1]
     q, k = _rand((T, Hq, d), 4), _rand((T, Hkv, d), 5)
     scale = 1.0 / math.sqrt(d)
@@ -96,7 +98,7 @@ def test_pooled_score_is_mean_of_raw_block_scores():
                     tot, cnt = 0.0, 0
                     for i in range(cu[b] + I * block, cu[b] + min(L, (I + 1) * block)):
                         for j in range(cu[b] + J * block, cu[b] + min(L, (J + 1) * block)):
-                            tot += scale * sum(q[i, h, c] * k[j, h // 2, c] for c in range(d))
+                            tot += scale * sum(q[i, h, c] * k[j, h // G, c] for c in range(d))
                             cnt += 1
                     assert s[b][h, I, J] == pytest.approx(tot / cnt, abs=1e-12)
 
@@ -150,9 +152,11 @@ def test_row_max_always_kept_and_alpha_limits(alpha):
         assert (keep.sum(axis=-1) == 1).all()
     if alpha == 1e-30:  # scores of std 3 span far less than ln(1e30) = 69: all kept
         assert np.array_equal(keep, np.broadcast_to(tri, keep.shape))
-    # softmax is shift invariant: adding a constant to a row changes nothing
-    keep2 = O.block_keep(s + 7.5, alpha, force_first=False, force_diag=False)
-    assert np.array_equal(keep, keep2)
+    # softmax is shift invariant: adding a constant to a row changes nothing, even a constant
+    # far past the range of exp (a softmax that does not subtract the row max overflows there)
+    for shift in (7.5, 800.0, -800.0):
+        keep2 = O.block_keep(s + shift, alpha, force_first=False, force_diag=False)
+        assert np.array_equal(keep, keep2)
 
 
 def test_masked_blocks_contribute_exactly_zero():
@@ -222,11 +226,12 @@ def test_per_head_scale_equals_prescaled_values():
     """e4m3 inputs enter as codes times a per-head scale; the product of a 4-bit code
     and a float32 scale is exact in float64, so scaling inside equals scaling outside."""
     cu = [0, 40]
-    T, Hq, Hkv, d, block = 40, 2, 1, 8, 8
+    T, Hq, Hkv, d, block = 40, 6, 2, 8, 8
     rng = np.random.Generator(np.random.PCG64(16))
     codes = lambda s: rng.integers(-16, 17, size=s).astype(np.float64) * 0.5
     q, k, v = codes((T, Hq, d)), codes((T, Hkv, d)), codes((T, Hkv, d))
-    qs, ks, vs = np.array([0.013, 0.25]), np.array([0.031]), np.array([0.7])
+    qs = np.array([0.013, 0.25, 0.5, 0.0625, 0.125, 2.0])
+    ks, vs = np.array([0.031, 0.375]), np.array([0.7, 0.0078125])
     scale = 1.0 / math.sqrt(d)
     a = O.pool_blocks(q, block, cu, scale=qs)
     b = O.pool_blocks(q * qs[None, :, None], block, cu)
@@ -330,3 +335,30 @@ def test_empty_request_contributes_nothing():
             assert O.keep_ratio(sc[1]).shape == (H, 0, 0)
         outs.append(O.masked_causal_attention(q, k, v, keeps, cu, B, 0.3)[0])
     assert np.array_equal(outs[0], outs[1])
+
+
+def test_chunked_request_without_new_queries_has_no_query_block():
+    """A request with cached keys but no new queries (q_len = 0, kv_len not a multiple of the
+    block) holds no query block: the batch with it gives the other requests exactly what the
+    batch without it gives, with the same pooled query rows."""
+    block, Hq, Hkv, d = 16, 2, 1, 8
+    scale = 1.0 / math.sqrt(d)
+    k0, k2, kx = _rand((70, Hkv, d), 51), _rand((33, Hkv, d), 52), _rand((37, Hkv, d), 53)
+    v0, v2, vx = _rand((70, Hkv, d), 54), _rand((33, Hkv, d), 55), _rand((37, Hkv, d), 56)
+    q = _rand((40, Hq, d), 57)                        # 30 new queries, then 10
+    runs = []
+    for kv_lens, q_lens, k, v in (([70, 37, 33], [30, 0, 10], np.concatenate([k0, kx, k2]),
+                                   np.concatenate([v0, vx, v2])),
+                                  ([70, 33], [30, 10], np.concatenate([k0, k2]),
+                                   np.concatenate([v0, v2]))):
+        ck = np.cumsum([0] + kv_lens).tolist()
+        cq = np.cumsum([0] + q_lens).tolist()
+        info, _ = O.query_blocks(cq, ck, block)
+        qp = O.pool_query_blocks(q, block, cq, ck)
+        sc = O.block_scores(qp, O.pool_blocks(k, block, ck), cq, block, scale, cu_k=ck)
+        keeps = [O.block_keep(x, 0.2, row0=info[b][1]) for b, x in enumerate(sc)]
+        runs.append((qp, *O.masked_causal_attention(q, k, v, keeps, cq, block, scale, cu_k=ck)))
+    (qp1, o1, l1), (qp2, o2, l2) = runs
+    assert qp1.shape == qp2.shape and np.array_equal(qp1, qp2)
+    assert np.isfinite(o1).all()
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
