@@ -162,8 +162,9 @@ int check_paging(const int32_t* page_table, int page_size, int max_pages, int nu
                  int block) {
   if (page_table &&
       (page_size < 16 || page_size % 16 || block % page_size || max_pages < 1 || num_pages < 1))
-    return fail(FP_ERR_INVALID_ARG, "page_size %d must be a multiple of 16 dividing block %d",
-                page_size, block);
+    return fail(FP_ERR_INVALID_ARG,
+                "page_size %d must be a multiple of 16 dividing block %d, and max_pages (%d) "
+                "and num_pages (%d) at least 1", page_size, block, max_pages, num_pages);
   return FP_OK;
 }
 

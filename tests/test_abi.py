@@ -51,6 +51,79 @@ def test_attention_rejects_bad_arguments(over, code):
     assert fp.library().fp_last_error_string()
 
 
+@pytest.mark.parametrize("over,code,msg", [
+    (dict(qs=16), -1, b"no scales"),                  # bf16 with a scale pointer
+    (dict(cu=16), -1, b"both given or both NULL"),    # one prefix-sum array without the other
+    (dict(T=-1, tb=0, mb=0), -1, b"negative"),
+    (dict(mb=3), -1, b"max_blocks must equal"),       # one sequence: max_blocks = total_blocks
+    (dict(Hq=0), -1, b"multiple of Hkv"),
+    (dict(out=None), -1, b"null pointer"),
+    (dict(ws=None), -1, b"null pointer"),
+    (dict(d=64, block=64, T=128, tb=2, mb=2, dtype=1, qs=16, ks=16, vs=16), -2, b"e4m3"),
+])
+def test_attention_error_messages(over, code, msg):
+    assert _bad_attn(**over) == code
+    assert msg in fp.library().fp_last_error_string()
+
+
+def _bad_paged(**over):
+    """A well-formed paged attention call with fake pointers (host validation only)."""
+    a = dict(q=16, k=16, v=16, dtype=0, qs=None, ks=None, vs=None, cu=16, cb=16, batch=2,
+             T=300, tb=3, mb=2, Hq=8, Hkv=2, d=128, block=128, pt=16, ps=64, mp=4, npg=8,
+             scale=0.1, cnt=16, idx=16, out=16, lse=None, ws=256, stream=None)
+    a.update(over)
+    return fp.library().fp_sparse_prefill_attn_paged(*a.values())
+
+
+@pytest.mark.parametrize("over,msg", [
+    (dict(pt=None), b"page table"),
+    (dict(cu=None, cb=None, batch=1, T=256, tb=2, mb=2), b"prefix sums"),
+    (dict(ps=48), b"page_size 48"),
+    (dict(ps=256), b"page_size 256"),                 # larger than the block
+    (dict(npg=0), b"num_pages (0)"),
+    (dict(mp=0), b"max_pages (0)"),
+])
+def test_paged_attention_rejects_bad_paging(over, msg):
+    assert _bad_paged(**over) == -1
+    assert msg in fp.library().fp_last_error_string()
+
+
+@pytest.mark.parametrize("args,code,msg", [
+    # (q_pool, k_pool, split, cu_blocks, batch, total_blocks, max_blocks, Hq, Hkv, d, alpha)
+    ((16, 16, None, None, 0, 4, 4, 8, 2, 128, 0.1), -1, b"batch"),
+    ((16, 16, None, None, 1, 4, 5, 8, 2, 128, 0.1), -1, b"max_blocks must equal"),
+    ((16, 16, None, None, 1, 4, 4, 6, 4, 128, 0.1), -1, b"multiple of Hkv"),
+    ((16, 16, None, None, 1, 4, 4, 8, 2, 96, 0.1), -2, b"head dim 96"),
+    ((8, 16, None, None, 1, 4, 4, 8, 2, 128, 0.1), -1, b"16-byte aligned"),
+    ((16, 16, 8, None, 1, 4, 4, 8, 2, 128, 0.1), -1, b"16-byte aligned"),
+    ((16, 16, None, None, 1, 4, 4, 8, 2, 128, float("nan")), -1, b"alpha"),
+    ((16, 16, None, None, 1, 4, 4, 8, 2, 128, -0.5), -1, b"alpha"),
+])
+def test_mask_error_messages(args, code, msg):
+    lib = fp.library()
+    rc = lib.fp_build_block_mask(*args, 0.1, 3, None, 16, 16, None)
+    assert rc == code
+    assert msg in lib.fp_last_error_string()
+
+
+def test_noalloc_refuses_problems_past_its_scratch():
+    """(Hq + Hkv) * total_blocks * d above 8 Mi floats: refused with a message, before any
+    CUDA call (this runs without a GPU)."""
+    lib = fp.library()
+    T = 2048 * 128
+    rc = lib.fp_pool_and_mask_noalloc(16, 16, 0, None, None, None, None, 1, T, 2048, 2048, 32, 8,
+                                      128, 128, None, 0, 0, 0, 0.1, 0.1, 3, None, 16, 16, None)
+    assert rc == -1
+    assert b"static scratch" in lib.fp_last_error_string()
+
+
+def test_debug_hook_and_status_reject_bad_arguments():
+    lib = fp.library()
+    assert lib.fp_debug_skip_k_load(-1) == -1
+    assert lib.fp_check_status(None, None) == -1
+    assert b"workspace" in lib.fp_last_error_string()
+
+
 def test_mask_rejects_alpha_out_of_range():
     lib = fp.library()
     rc = lib.fp_build_block_mask(16, 16, None, None, 1, 4, 4, 8, 2, 128, 1.5, 0.1, 3, None, 16,
