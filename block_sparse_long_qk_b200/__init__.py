@@ -139,6 +139,54 @@ def _same_dtype(*ts):
                         + ", ".join(str(t.dtype) for t in ts))
 
 
+def _expect(t, name, shape=None, dtype=None, min_numel=None):
+    """Host-side check of a tensor the kernels read or write: the C ABI receives only a
+    pointer and the sizes derived from the other arguments, so a tensor smaller than those
+    sizes would be read or written past its end on the GPU. Refused here instead."""
+    if t is None:
+        return
+    if shape is not None and tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name}: expected shape {tuple(int(x) for x in shape)}, got "
+                         f"{tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name}: expected at least {int(min_numel)} elements, got "
+                         f"{t.numel()}")
+
+
+def _expect_heads(q, k, name_k="k"):
+    """Q [T, Hq, d] and K [*, Hkv, d]: same head dim, Hq a multiple of Hkv."""
+    if q.dim() != 3:
+        raise ValueError(f"q: expected [tokens, Hq, d], got shape {tuple(q.shape)}")
+    if k.dim() < 3 or k.shape[-1] != q.shape[-1]:
+        raise ValueError(f"{name_k}: expected head dim {q.shape[-1]}, got shape "
+                         f"{tuple(k.shape)}")
+    if q.shape[1] % k.shape[-2] != 0:
+        raise ValueError(f"Hq = {q.shape[1]} is not a multiple of Hkv = {k.shape[-2]}")
+
+
+def _expect_scales(q_scale, k_scale, v_scale, Hq, Hkv):
+    _expect(q_scale, "q_scale", (Hq,), torch.float32)
+    _expect(k_scale, "k_scale", (Hkv,), torch.float32)
+    _expect(v_scale, "v_scale", (Hkv,), torch.float32)
+
+
+def _expect_paged(paged, d, batch_size, need_v):
+    """Caches [num_pages, page_size, Hkv, d] and an int32 page table with a row per request."""
+    kc = paged.k_cache
+    if kc.dim() != 4 or kc.shape[-1] != d:
+        raise ValueError(f"k_cache: expected [num_pages, page_size, Hkv, {d}], got shape "
+                         f"{tuple(kc.shape)}")
+    if need_v:
+        _expect(paged.v_cache, "v_cache", kc.shape)
+    pt = paged.page_table
+    if pt.dim() != 2 or pt.shape[0] < batch_size:
+        raise ValueError(f"page_table: expected [batch >= {batch_size}, max_pages], got shape "
+                         f"{tuple(pt.shape)}")
+    _expect(pt, "page_table", dtype=torch.int32)
+
+
 def _dtype_code(t):
     if t.dtype == torch.bfloat16:
         return FP_DTYPE_BF16
@@ -225,17 +273,30 @@ def _batch_for(q, block, batch):
     return batch
 
 
+def _expect_tokens(b, T):
+    if b.total_tokens != T:
+        raise ValueError(f"the batch holds {b.total_tokens} tokens but q has {T} rows")
+
+
 def pool_qk(q, k, block=128, *, batch: Batch | None = None, q_scale=None, k_scale=None,
             paged: PagedKV | None = None, k_split_out=None):
     """Block means of Q [T,Hq,d] and K [T,Hkv,d] (or the paged K cache) -> float32
     q_pool [Hq, nblk, d], k_pool [Hkv, nblk, d]. With ``k_split_out`` (bf16 tensor of
     ``k_split_shape``) the kernel also writes the hi / lo bf16 split of k_pool there, which
     ``build_block_mask(k_split=...)`` then loads instead of converting."""
-    T, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
+    _expect_heads(q, kk, "k_cache" if paged is not None else "k")
+    T, Hq, d = q.shape
     _same_dtype(q, kk)
     Hkv = kk.shape[-2]
     b = _batch_for(q, block, batch)
+    _expect_tokens(b, T)
+    if paged is not None:
+        _expect_paged(paged, d, b.size, need_v=False)
+    else:
+        _expect(k, "k", (T, Hkv, d))
+    _expect_scales(q_scale, k_scale, None, Hq, Hkv)
+    _expect(k_split_out, "k_split_out", k_split_shape(Hkv, b.total_blocks, d), torch.bfloat16)
     q_pool = torch.empty((Hq, b.total_blocks, d), dtype=torch.float32, device=q.device)
     k_pool = torch.empty((Hkv, b.total_blocks, d), dtype=torch.float32, device=q.device)
     cu, cb = b._ptrs()
@@ -262,9 +323,14 @@ def build_block_mask(q_pool, k_pool, alpha=0.1, *, block=128, batch: Batch | Non
     [Hq, nblk, max_blocks] int32)."""
     Hq, nblk, d = q_pool.shape
     Hkv = k_pool.shape[0]
+    _expect(q_pool, "q_pool", dtype=torch.float32)
+    _expect(k_pool, "k_pool", (Hkv, nblk, d), torch.float32)
+    _expect(k_split, "k_split", k_split_shape(Hkv, nblk, d), torch.bfloat16)
     if batch is None:
         batch = Batch.make((nblk * block,), block, q_pool.device)
         batch = dataclasses.replace(batch, total_blocks=nblk, max_blocks=nblk)
+    elif batch.total_blocks != nblk:
+        raise ValueError(f"the batch holds {batch.total_blocks} blocks but q_pool has {nblk}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     words = (batch.max_blocks + 31) // 32
@@ -281,14 +347,29 @@ def build_block_mask(q_pool, k_pool, alpha=0.1, *, block=128, batch: Batch | Non
     return bits, kv_cnt, kv_idx
 
 
+def _expect_lists(kv_cnt, kv_idx, Hq, nblk, max_blocks):
+    """kv_cnt int32 [Hq, nblk] and kv_idx int32 [Hq, nblk, max_blocks] (or larger buffers)."""
+    if kv_cnt is None or kv_idx is None:
+        raise ValueError("kv_cnt and kv_idx are required")
+    _expect(kv_cnt, "kv_cnt", dtype=torch.int32, min_numel=Hq * nblk)
+    _expect(kv_idx, "kv_idx", dtype=torch.int32, min_numel=Hq * nblk * max_blocks)
+
+
 def sparse_prefill_attn(q, k, v, kv_cnt, kv_idx, block=128, *, batch: Batch | None = None,
                         scale=None, q_scale=None, k_scale=None, v_scale=None,
                         return_lse=False, out=None, ws=None):
     """Causal attention over the kept KV blocks -> (out bf16 [T,Hq,d], lse [Hq,T] or None)."""
     _same_dtype(q, k, v)
+    _expect_heads(q, k)
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     b = _batch_for(q, block, batch)
+    _expect_tokens(b, T)
+    _expect(k, "k", (T, Hkv, d))
+    _expect(v, "v", (T, Hkv, d))
+    _expect_lists(kv_cnt, kv_idx, Hq, b.total_blocks, b.max_blocks)
+    _expect_scales(q_scale, k_scale, v_scale, Hq, Hkv)
+    _expect(out, "out", (T, Hq, d), torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -308,8 +389,14 @@ def sparse_prefill_attn_paged(q, paged: PagedKV, kv_cnt, kv_idx, batch: Batch, *
                               return_lse=False, out=None, ws=None):
     """Same as ``sparse_prefill_attn`` with K/V read through the page table."""
     _same_dtype(q, paged.k_cache, paged.v_cache)
+    _expect_heads(q, paged.k_cache, "k_cache")
     T, Hq, d = q.shape
     Hkv = paged.k_cache.shape[2]
+    _expect_tokens(batch, T)
+    _expect_paged(paged, d, batch.size, need_v=True)
+    _expect_lists(kv_cnt, kv_idx, Hq, batch.total_blocks, batch.max_blocks)
+    _expect_scales(q_scale, k_scale, v_scale, Hq, Hkv)
+    _expect(out, "out", (T, Hq, d), torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -360,11 +447,18 @@ def pool_and_mask_noalloc(q, k, alpha=0.1, block=128, *, batch: Batch | None = N
     """``pool_qk`` + ``build_block_mask`` with the pooled means kept in the library's static
     device scratch (for callers that cannot allocate them). Returns (mask_bits or None,
     kv_cnt, kv_idx); the output tensors are allocated here by torch for convenience."""
-    T, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
+    _expect_heads(q, kk, "k_cache" if paged is not None else "k")
+    T, Hq, d = q.shape
     _same_dtype(q, kk)
     Hkv = kk.shape[-2]
     b = _batch_for(q, block, batch)
+    _expect_tokens(b, T)
+    if paged is not None:
+        _expect_paged(paged, d, b.size, need_v=False)
+    else:
+        _expect(k, "k", (T, Hkv, d))
+    _expect_scales(q_scale, k_scale, None, Hq, Hkv)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dev = q.device
@@ -438,14 +532,32 @@ class ChunkedBatch:
                 self.size)
 
 
+def _expect_chunk_rows(cb, q, k, v, paged, need_v):
+    """Q [total_q, Hq, d]; K and V [total_k, Hkv, d] or the caches of ``paged``."""
+    T, Hq, d = q.shape
+    if T != cb.total_q:
+        raise ValueError(f"the batch holds {cb.total_q} queries but q has {T} rows")
+    if paged is not None:
+        _expect_paged(paged, d, cb.size, need_v)
+    else:
+        Hkv = k.shape[-2]
+        _expect(k, "k", (cb.total_k, Hkv, d))
+        if need_v:
+            _expect(v, "v", (cb.total_k, Hkv, d))
+
+
 def pool_qk_chunked(q, k, cb: ChunkedBatch, *, q_scale=None, k_scale=None,
                     paged: PagedKV | None = None, k_split_out=None):
     """Block means for a chunked batch: q_pool [Hq, total_qblocks, d] over the queries each
     query block holds, k_pool [Hkv, total_kblocks, d] over all keys (cached prefix included)."""
-    _, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
+    _expect_heads(q, kk, "k_cache" if paged is not None else "k")
+    _, Hq, d = q.shape
     _same_dtype(q, kk)
     Hkv = kk.shape[-2]
+    _expect_chunk_rows(cb, q, k, None, paged, need_v=False)
+    _expect_scales(q_scale, k_scale, None, Hq, Hkv)
+    _expect(k_split_out, "k_split_out", k_split_shape(Hkv, cb.total_kblocks, d), torch.bfloat16)
     q_pool = torch.empty((Hq, cb.total_qblocks, d), dtype=torch.float32, device=q.device)
     k_pool = torch.empty((Hkv, cb.total_kblocks, d), dtype=torch.float32, device=q.device)
     pt = paged.page_table if paged is not None else None
@@ -464,6 +576,11 @@ def build_block_mask_chunked(q_pool, k_pool, cb: ChunkedBatch, alpha=0.1, *, sca
     kv_cnt [Hq, total_qblocks], kv_idx [Hq, total_qblocks, max_kblocks])."""
     Hq, nqb, d = q_pool.shape
     Hkv = k_pool.shape[0]
+    if nqb != cb.total_qblocks:
+        raise ValueError(f"the batch holds {cb.total_qblocks} query blocks but q_pool has {nqb}")
+    _expect(q_pool, "q_pool", dtype=torch.float32)
+    _expect(k_pool, "k_pool", (Hkv, cb.total_kblocks, d), torch.float32)
+    _expect(k_split, "k_split", k_split_shape(Hkv, cb.total_kblocks, d), torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dev = q_pool.device
@@ -484,11 +601,16 @@ def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
     """Attention of the chunk's queries over the kept KV blocks of the whole request ->
     (out bf16 [total_q, Hq, d], lse [Hq, total_q] or None). K/V are contiguous [total_k, Hkv,
     d] (``k``, ``v``) or the caches of ``paged``."""
-    T, Hq, d = q.shape
     kk = paged.k_cache if paged is not None else k
     vv = paged.v_cache if paged is not None else v
     _same_dtype(q, kk, vv)
+    _expect_heads(q, kk, "k_cache" if paged is not None else "k")
+    T, Hq, d = q.shape
     Hkv = kk.shape[-2]
+    _expect_chunk_rows(cb, q, k, v, paged, need_v=True)
+    _expect_lists(kv_cnt, kv_idx, Hq, cb.total_qblocks, cb.max_kblocks)
+    _expect_scales(q_scale, k_scale, v_scale, Hq, Hkv)
+    _expect(out, "out", (T, Hq, d), torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -511,6 +633,12 @@ def append_paged_kv(k_new, v_new, cb: ChunkedBatch, paged: PagedKV, *, ws=None):
     absolute positions (before the chunked prefill reads them)."""
     T, Hkv, d = k_new.shape
     _same_dtype(k_new, v_new, paged.k_cache, paged.v_cache)
+    if T != cb.total_q:
+        raise ValueError(f"the batch holds {cb.total_q} new rows but k_new has {T}")
+    _expect(v_new, "v_new", (T, Hkv, d))
+    _expect_paged(paged, d, cb.size, need_v=True)
+    if paged.k_cache.shape[2] != Hkv:
+        raise ValueError(f"k_cache holds {paged.k_cache.shape[2]} KV heads, k_new {Hkv}")
     ws = workspace(k_new.device) if ws is None else ws
     pt = paged.page_table
     _check(library().fp_append_paged_kv(
