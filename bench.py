@@ -34,6 +34,10 @@ from block_sparse_long_qk_b200 import synthetic as S  # noqa: E402
 
 METRIC = "128K prefill-attn ms/layer incl. mask build; executed TFLOPS & % of B200 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures (dense bf16 tensor rate, HBM3e bandwidth), reported beside the
+# measured denominators for context only.
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 7700.0
 
 
 def _peaks():
@@ -337,6 +341,7 @@ def run_native(args, world, rank, local):
     peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     if w.dtype == "e4m3":
         peak_t *= 2.0   # e4m3 dense rate = 2x bf16 (nominal ratio); no measured e4m3 peak
+    nominal_t = NOMINAL_BF16_TFLOPS * (2.0 if w.dtype == "e4m3" else 1.0)
     traffic = None
     tf = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if os.path.exists(tf):
@@ -349,7 +354,10 @@ def run_native(args, world, rank, local):
             "peak_source": f"{peak_src} bf16 sustained" + (" x2 (e4m3 nominal ratio)"
                                                           if w.dtype == "e4m3" else ""),
             "executed_tflops": round(executed / (attn_ms * 1e-3) / 1e12, 2),
-            "executed_frac": round(executed / (attn_ms * 1e-3) / 1e12 / peak_t, 4)}
+            "executed_frac": round(executed / (attn_ms * 1e-3) / 1e12 / peak_t, 4),
+            # the datasheet's dense figure, for context (2.25 PFLOP/s bf16, 4.5 e4m3)
+            "nominal_peak": nominal_t,
+            "frac_of_nominal": round(alg / (attn_ms * 1e-3) / 1e12 / nominal_t, 4)}
 
     # e2e: host (pinned) inputs -> device, the layer, output -> host, per step
     e2e = None
@@ -377,7 +385,9 @@ def run_native(args, world, rank, local):
                                             peaks["hbm_gbs"], 4),
                           "pool_bytes": pool_bytes,
                           "pool_frac_hbm": round(pool_bytes / (pool_ms * 1e-3) / 1e9 /
-                                                 peaks["hbm_gbs"], 4)},
+                                                 peaks["hbm_gbs"], 4),
+                          "frac_hbm_nominal": round(pm_bytes / ((pool_ms + mask_ms) * 1e-3) /
+                                                    1e9 / NOMINAL_HBM_GBS, 4)},
             "block_density": round(density, 5),
             "attn_tflop": {"algorithmic": round(alg / 1e12, 3),
                            "executed": round(executed / 1e12, 3)},
