@@ -33,7 +33,7 @@ __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_at
            "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "MASK_FP32", "header_symbols",
            "pool_and_mask_noalloc", "k_split_shape", "ChunkedBatch", "pool_qk_chunked",
            "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked",
-           "HostPipeline", "append_paged_kv", "GraphStep"]
+           "HostPipeline", "append_paged_kv", "GraphStep", "head_shard"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfpsparse.so")
@@ -51,9 +51,9 @@ _SIGNATURES = {
     "fp_last_error_string": (ctypes.c_char_p, []),
     "fp_workspace_size": (_sz, []),
     "fp_pool_qk": (_i, [_p, _p, _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i,
-                        _i, _p, _p, _p, _p]),
+                        _i, _p, _p, _p, _p, _p]),
     "fp_build_block_mask": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _f, _i, _p, _p,
-                                 _p, _p]),
+                                 _p, _p, _p]),
     "fp_sparse_prefill_attn": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i,
                                     _i, _i, _i, _f, _p, _p, _p, _p, _p, _p]),
     "fp_sparse_prefill_attn_paged": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _i, _i, _i, _i,
@@ -61,12 +61,13 @@ _SIGNATURES = {
                                           _p, _p]),
     "fp_check_status": (_i, [_p, _p]),
     "fp_debug_skip_k_load": (_i, [_i]),
+    "fp_debug_skip_mask_load": (_i, [_i]),
     "fp_pool_and_mask_noalloc": (_i, [_p, _p, _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
                                       _i, _p, _i, _i, _i, _f, _f, _i, _p, _p, _p, _p]),
     "fp_pool_qk_chunked": (_i, [_p, _p, _i, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i,
-                                _i, _i, _p, _i, _i, _i, _p, _p, _p, _p]),
+                                _i, _i, _p, _i, _i, _i, _p, _p, _p, _p, _p]),
     "fp_build_block_mask_chunked": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i,
-                                         _i, _i, _f, _f, _i, _p, _p, _p, _p]),
+                                         _i, _i, _f, _f, _i, _p, _p, _p, _p, _p]),
     "fp_append_paged_kv": (_i, [_p, _p, _i, _p, _p, _i, _i, _i, _i, _p, _i, _i, _i, _p, _p, _p,
                                 _p]),
     "fp_sparse_prefill_attn_chunked": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _i, _i,
@@ -242,6 +243,23 @@ class PagedKV:
         return self.k_cache.shape[1]
 
 
+def head_shard(Hq, Hkv, rank, world):
+    """The heads that rank ``rank`` of ``world`` owns when one layer is split by KV-head group:
+    (query-head slice, KV-head slice). A query head reads only its own KV head in all three
+    stages (pooled scores, mask and attention), so each rank runs the whole path on its slice
+    with no exchange between ranks. Groups are dealt as evenly as they go: the first
+    Hkv % world ranks take one group more. At most Hkv ranks."""
+    if Hq <= 0 or Hkv <= 0 or Hq % Hkv:
+        raise ValueError(f"Hq ({Hq}) must be a positive multiple of Hkv ({Hkv})")
+    if not 1 <= world <= Hkv or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of {world}: a head split needs 1 <= world <= Hkv ({Hkv})")
+    base, extra = divmod(Hkv, world)
+    g0 = rank * base + min(rank, extra)
+    g1 = g0 + base + (1 if rank < extra else 0)
+    G = Hq // Hkv
+    return slice(g0 * G, g1 * G), slice(g0, g1)
+
+
 _workspaces = {}
 
 
@@ -258,8 +276,8 @@ def workspace(device):
 
 
 def check_status(device=None, ws=None):
-    """Waits for the current stream and raises if an attention launch recorded a pipeline
-    timeout or an out-of-range index since the last check."""
+    """Waits for the current stream and raises if a launch on the workspace recorded a
+    pipeline timeout, an out-of-range index or inconsistent prefix sums since the last check."""
     if ws is None:
         ws = workspace(device if device is not None else torch.device("cuda"))
     _check(library().fp_check_status(_ptr(ws), _stream(ws.device)))
@@ -279,7 +297,7 @@ def _expect_tokens(b, T):
 
 
 def pool_qk(q, k, block=128, *, batch: Batch | None = None, q_scale=None, k_scale=None,
-            paged: PagedKV | None = None, k_split_out=None):
+            paged: PagedKV | None = None, k_split_out=None, ws=None):
     """Block means of Q [T,Hq,d] and K [T,Hkv,d] (or the paged K cache) -> float32
     q_pool [Hq, nblk, d], k_pool [Hkv, nblk, d]. With ``k_split_out`` (bf16 tensor of
     ``k_split_shape``) the kernel also writes the hi / lo bf16 split of k_pool there, which
@@ -307,7 +325,8 @@ def pool_qk(q, k, block=128, *, batch: Batch | None = None, q_scale=None, k_scal
         _ptr(q), _ptr(kk), _dtype_code(q), _ptr(q_scale), _ptr(k_scale), cu, cb, b.size, T,
         b.total_blocks, Hq, Hkv, d, block, _ptr(pt), paged.page_size if paged else 0,
         pt.shape[1] if pt is not None else 0, kk.shape[0] if pt is not None else 0,
-        _ptr(q_pool), _ptr(k_pool), _ptr(k_split_out), _stream(q.device)))
+        _ptr(q_pool), _ptr(k_pool), _ptr(k_split_out),
+        _ptr(workspace(q.device) if ws is None else ws), _stream(q.device)))
     return q_pool, k_pool
 
 
@@ -317,7 +336,8 @@ def k_split_shape(Hkv, total_blocks, d):
 
 
 def build_block_mask(q_pool, k_pool, alpha=0.1, *, block=128, batch: Batch | None = None,
-                     scale=None, flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True, k_split=None):
+                     scale=None, flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True, k_split=None,
+                     ws=None):
     """Max-based dynamic threshold on the pooled block scores -> (mask_bits or None
     [Hq, nblk, words] uint32 viewed as int32, kv_cnt [Hq, nblk] int32, kv_idx
     [Hq, nblk, max_blocks] int32)."""
@@ -343,7 +363,7 @@ def build_block_mask(q_pool, k_pool, alpha=0.1, *, block=128, batch: Batch | Non
         _ptr(q_pool), _ptr(k_pool), _ptr(k_split), cb, batch.size, nblk, batch.max_blocks, Hq,
         Hkv, d,
         float(alpha), float(scale), int(flags), _ptr(bits), _ptr(kv_cnt), _ptr(kv_idx),
-        _stream(dev)))
+        _ptr(workspace(dev) if ws is None else ws), _stream(dev)))
     return bits, kv_cnt, kv_idx
 
 
@@ -547,7 +567,7 @@ def _expect_chunk_rows(cb, q, k, v, paged, need_v):
 
 
 def pool_qk_chunked(q, k, cb: ChunkedBatch, *, q_scale=None, k_scale=None,
-                    paged: PagedKV | None = None, k_split_out=None):
+                    paged: PagedKV | None = None, k_split_out=None, ws=None):
     """Block means for a chunked batch: q_pool [Hq, total_qblocks, d] over the queries each
     query block holds, k_pool [Hkv, total_kblocks, d] over all keys (cached prefix included)."""
     kk = paged.k_cache if paged is not None else k
@@ -566,12 +586,13 @@ def pool_qk_chunked(q, k, cb: ChunkedBatch, *, q_scale=None, k_scale=None,
         cb.total_q, cb.total_k, cb.total_qblocks, cb.total_kblocks, Hq, Hkv, d, cb.block,
         _ptr(pt), paged.page_size if paged else 0, pt.shape[1] if pt is not None else 0,
         kk.shape[0] if pt is not None else 0, _ptr(q_pool), _ptr(k_pool), _ptr(k_split_out),
-        _stream(q.device)))
+        _ptr(workspace(q.device) if ws is None else ws), _stream(q.device)))
     return q_pool, k_pool
 
 
 def build_block_mask_chunked(q_pool, k_pool, cb: ChunkedBatch, alpha=0.1, *, scale=None,
-                             flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True, k_split=None):
+                             flags=FORCE_FIRST | FORCE_DIAG, mask_bits=True, k_split=None,
+                             ws=None):
     """Threshold for a chunked batch -> (mask_bits or None [Hq, total_qblocks, words],
     kv_cnt [Hq, total_qblocks], kv_idx [Hq, total_qblocks, max_kblocks])."""
     Hq, nqb, d = q_pool.shape
@@ -591,7 +612,8 @@ def build_block_mask_chunked(q_pool, k_pool, cb: ChunkedBatch, alpha=0.1, *, sca
     _check(library().fp_build_block_mask_chunked(
         _ptr(q_pool), _ptr(k_pool), _ptr(k_split), *cb._args(), cb.total_qblocks,
         cb.total_kblocks, cb.max_kblocks, Hq, Hkv, d, cb.block, float(alpha), float(scale),
-        int(flags), _ptr(bits), _ptr(kv_cnt), _ptr(kv_idx), _stream(dev)))
+        int(flags), _ptr(bits), _ptr(kv_cnt), _ptr(kv_idx),
+        _ptr(workspace(dev) if ws is None else ws), _stream(dev)))
     return bits, kv_cnt, kv_idx
 
 

@@ -1,5 +1,6 @@
 // extern "C" entry points of libfpsparse.so: argument checks, then one kernel launch each.
 // Declarations and the contract of every call are in include/fpsparse.h.
+#include <limits.h>
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -15,6 +16,7 @@ namespace {
 
 thread_local std::string g_err;
 thread_local int g_fault_skip_k = -1;  // one-shot test hook for the next attention call
+thread_local int g_fault_skip_mask = -1;  // one-shot test hook for the next mask call
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -31,6 +33,13 @@ int cuda_fail(cudaError_t e, const char* what) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The workspace holds the status word; NULL is allowed where the call says so.
+int check_workspace(const void* workspace) {
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  return FP_OK;
+}
 
 // The small index arrays (prefix sums, page tables) are the arguments most easily left in
 // host memory by a caller; a kernel reading one would fault the GPU. Each non-NULL one must
@@ -116,7 +125,7 @@ int set_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int fp_version(void) { return 110; }
+int fp_version(void) { return 200; }
 
 const char* fp_last_error_string(void) { return g_err.c_str(); }
 
@@ -171,8 +180,9 @@ int check_paging(const int32_t* page_table, int page_size, int max_pages, int nu
 int pool_impl(const void* q, const void* k, int dtype, const float* q_scale,
               const float* k_scale, const fp::Seqs& s, int Hq, int Hkv, int d,
               const int32_t* k_page_table, int page_size, int max_pages, int num_pages,
-              float* q_pool, float* k_pool, void* k_pool_split, void* stream) {
+              float* q_pool, float* k_pool, void* k_pool_split, void* workspace, void* stream) {
   if (!q || !k || !q_pool || !k_pool) return fail(FP_ERR_INVALID_ARG, "null tensor pointer");
+  if (check_workspace(workspace)) return FP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool) ||
       !aligned16(k_pool_split))
     return fail(FP_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
@@ -183,9 +193,11 @@ int pool_impl(const void* q, const void* k, int dtype, const float* q_scale,
   if (s.total_kb == 0) return FP_OK;
   rc = check_device_arrays(stream, {{s.cu_q, "cu_q / cu_seqlens"},
                                     {s.cu_qb, "cu_qblocks / cu_blocks"}, {s.cu_k, "cu_k"},
-                                    {s.cu_kb, "cu_kblocks"}, {k_page_table, "k_page_table"}});
+                                    {s.cu_kb, "cu_kblocks"}, {k_page_table, "k_page_table"},
+                                    {workspace, "workspace"}});
   if (rc) return rc;
   fp::PoolArgs a{};
+  a.status = static_cast<uint32_t*>(workspace);
   a.q = static_cast<const uint8_t*>(q);
   a.k = static_cast<const uint8_t*>(k);
   a.q_scale = q_scale;
@@ -207,8 +219,12 @@ int pool_impl(const void* q, const void* k, int dtype, const float* q_scale,
 
 int mask_impl(const float* q_pool, const float* k_pool, const void* k_pool_split,
               const fp::Seqs& s, int Hq, int Hkv, int d, float alpha, float scale, int flags,
-              uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* stream) {
+              uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* workspace,
+              void* stream) {
+  const int skip_chunk = g_fault_skip_mask;
+  g_fault_skip_mask = -1;
   if (!q_pool || !k_pool || !kv_cnt || !kv_idx) return fail(FP_ERR_INVALID_ARG, "null pointer");
+  if (check_workspace(workspace)) return FP_ERR_INVALID_ARG;
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv)
     return fail(FP_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", Hq, Hkv);
   if (d != 64 && d != 128) return fail(FP_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
@@ -217,7 +233,8 @@ int mask_impl(const float* q_pool, const float* k_pool, const void* k_pool_split
     return fail(FP_ERR_INVALID_ARG, "pooled tensors must be 16-byte aligned");
   if (s.total_qb == 0) return FP_OK;
   int rc = check_device_arrays(stream, {{s.cu_q, "cu_q"}, {s.cu_qb, "cu_qblocks / cu_blocks"},
-                                        {s.cu_k, "cu_k"}, {s.cu_kb, "cu_kblocks"}});
+                                        {s.cu_k, "cu_k"}, {s.cu_kb, "cu_kblocks"},
+                                        {workspace, "workspace"}});
   if (rc) return rc;
   const int G = Hq / Hkv;
   const int nb = fp::mask_blocks_per_cta(G, d, s.max_kb);
@@ -232,6 +249,8 @@ int mask_impl(const float* q_pool, const float* k_pool, const void* k_pool_split
   a.mask_bits = mask_bits;
   a.kv_cnt = kv_cnt;
   a.kv_idx = kv_idx;
+  a.status = static_cast<uint32_t*>(workspace);
+  a.fault_skip_chunk = skip_chunk;
   a.s = s;
   a.Hq = Hq;
   a.Hkv = Hkv;
@@ -254,8 +273,7 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
     return fail(FP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(FP_ERR_INVALID_ARG, "Q, K, V and out must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(FP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (check_workspace(workspace)) return FP_ERR_INVALID_ARG;
   if (dtype == FP_DTYPE_E4M3 && !(d == 128 && s.block == 128))
     return fail(FP_ERR_UNSUPPORTED, "e4m3 attention supports d = 128, block = 128");
   int rc = check_paging(page_table, page_size, max_pages, num_pages, s.block);
@@ -313,7 +331,8 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
                const float* k_scale, const int32_t* cu_seqlens, const int32_t* cu_blocks,
                int batch, int total_tokens, int total_blocks, int Hq, int Hkv, int d,
                int block, const int32_t* k_page_table, int page_size, int max_pages,
-               int num_pages, float* q_pool, float* k_pool, void* k_pool_split, void* stream) {
+               int num_pages, float* q_pool, float* k_pool, void* k_pool_split,
+               void* workspace, void* stream) {
   g_err.clear();
   int rc = check_common(dtype, q_scale, k_scale, nullptr, false, cu_seqlens, cu_blocks, batch,
                         total_tokens, total_blocks, Hq, Hkv, d, block);
@@ -322,13 +341,14 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
                    plain_seqs(cu_seqlens, cu_blocks, batch, total_tokens, total_blocks,
                               total_blocks, block),
                    Hq, Hkv, d, k_page_table, page_size, max_pages, num_pages, q_pool, k_pool,
-                   k_pool_split, stream);
+                   k_pool_split, workspace, stream);
 }
 
 int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_pool_split,
                         const int32_t* cu_blocks, int batch, int total_blocks, int max_blocks,
                         int Hq, int Hkv, int d, float alpha, float scale, int flags,
-                        uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* stream) {
+                        uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* workspace,
+                        void* stream) {
   g_err.clear();
   if (batch < 1 || (batch > 1 && !cu_blocks))
     return fail(FP_ERR_INVALID_ARG, "batch > 1 needs cu_blocks");
@@ -341,7 +361,7 @@ int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_
   const fp::Seqs s = plain_seqs(cu_blocks, cu_blocks, batch, total_blocks, total_blocks,
                                 max_blocks, 1);
   return mask_impl(q_pool, k_pool, k_pool_split, s, Hq, Hkv, d, alpha, scale, flags, mask_bits,
-                   kv_cnt, kv_idx, stream);
+                   kv_cnt, kv_idx, workspace, stream);
 }
 
 int fp_sparse_prefill_attn(const void* q, const void* k, const void* v, int dtype,
@@ -412,7 +432,7 @@ int fp_pool_qk_chunked(const void* q, const void* k, int dtype, const float* q_s
                        int total_k, int total_qblocks, int total_kblocks, int Hq, int Hkv,
                        int d, int block, const int32_t* k_page_table, int page_size,
                        int max_pages, int num_pages, float* q_pool, float* k_pool,
-                       void* k_pool_split, void* stream) {
+                       void* k_pool_split, void* workspace, void* stream) {
   g_err.clear();
   int rc = check_common(dtype, q_scale, k_scale, nullptr, false, cu_q, cu_qblocks, batch,
                         total_q, total_qblocks, Hq, Hkv, d, block);
@@ -420,11 +440,13 @@ int fp_pool_qk_chunked(const void* q, const void* k, int dtype, const float* q_s
   rc = check_chunked(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, total_q, total_k, total_qblocks,
                      total_kblocks, total_kblocks > 0 ? 1 : 0);
   if (rc) return rc;
+  // The pool kernel needs no per-row list length: any request's block count is at most
+  // total_kblocks.
   return pool_impl(q, k, dtype, q_scale, k_scale,
                    chunked_seqs(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, total_q, total_k,
-                                total_qblocks, total_kblocks, 0, block),
+                                total_qblocks, total_kblocks, total_kblocks, block),
                    Hq, Hkv, d, k_page_table, page_size, max_pages, num_pages, q_pool, k_pool,
-                   k_pool_split, stream);
+                   k_pool_split, workspace, stream);
 }
 
 int fp_build_block_mask_chunked(const float* q_pool, const float* k_pool,
@@ -434,17 +456,20 @@ int fp_build_block_mask_chunked(const float* q_pool, const float* k_pool,
                                 int total_kblocks, int max_kblocks, int Hq, int Hkv, int d,
                                 int block, float alpha, float scale, int flags,
                                 uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx,
-                                void* stream) {
+                                void* workspace, void* stream) {
   g_err.clear();
   if (block != 64 && block != 128)
     return fail(FP_ERR_UNSUPPORTED, "block %d (supported: 64, 128)", block);
   int rc = check_chunked(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, 0, 0, total_qblocks,
                          total_kblocks, max_kblocks);
   if (rc) return rc;
+  // The mask reads no token rows, and this call is not given the token totals: the device-side
+  // checks of the prefix sums bound the rows by INT_MAX and the blocks by the totals passed.
   return mask_impl(q_pool, k_pool, k_pool_split,
-                   chunked_seqs(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, 0, 0, total_qblocks,
-                                total_kblocks, max_kblocks, block),
-                   Hq, Hkv, d, alpha, scale, flags, mask_bits, kv_cnt, kv_idx, stream);
+                   chunked_seqs(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, INT_MAX, INT_MAX,
+                                total_qblocks, total_kblocks, max_kblocks, block),
+                   Hq, Hkv, d, alpha, scale, flags, mask_bits, kv_cnt, kv_idx, workspace,
+                   stream);
 }
 
 int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, int dtype,
@@ -486,8 +511,7 @@ int fp_append_paged_kv(const void* k_new, const void* v_new, int dtype, const in
     return fail(FP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
     return fail(FP_ERR_INVALID_ARG, "K/V rows and caches must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(FP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (check_workspace(workspace)) return FP_ERR_INVALID_ARG;
   if (page_size < 1 || max_pages < 1 || num_pages < 1)
     return fail(FP_ERR_INVALID_ARG, "page_size, max_pages and num_pages must be >= 1");
   if (total_q == 0) return FP_OK;
@@ -520,6 +544,13 @@ int fp_debug_skip_k_load(int union_block) {
   return FP_OK;
 }
 
+int fp_debug_skip_mask_load(int chunk) {
+  g_err.clear();
+  if (chunk < 0) return fail(FP_ERR_INVALID_ARG, "chunk index must be >= 0");
+  g_fault_skip_mask = chunk;
+  return FP_OK;
+}
+
 int fp_check_status(void* workspace, void* stream) {
   g_err.clear();
   if (!workspace) return fail(FP_ERR_INVALID_ARG, "null workspace");
@@ -534,9 +565,10 @@ int fp_check_status(void* workspace, void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
   }
   if (word & fp::kStatusTimeout)
-    return fail(FP_ERR_TIMEOUT, "a pipeline wait in the attention kernel timed out");
+    return fail(FP_ERR_TIMEOUT, "a pipeline wait in the mask or attention kernel timed out");
   if (word & fp::kStatusBadIndex)
-    return fail(FP_ERR_BAD_INDEX, "an index list or page table entry was out of range");
+    return fail(FP_ERR_BAD_INDEX, "an index list, page table entry or prefix sum was out of "
+                "range or inconsistent");
   return FP_OK;
 }
 

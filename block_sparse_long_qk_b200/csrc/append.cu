@@ -14,12 +14,14 @@ constexpr int kAppendThreads = 128;
 constexpr int kAppendRows = 8;  // new rows per CTA, their loads in flight together
 
 // Destination row of new row t in the cache, or -1 (and the status bit) when its page entry is
-// out of range.
+// out of range or the prefix sums of its request are inconsistent (q0 <= t < q1 and at most as
+// many new rows as keys).
 __device__ __forceinline__ long long append_dst_row(const AppendArgs& a, int t) {
   const int b = seqs_find(a.s.cu_q, a.s.batch, t);
   const int q0 = __ldg(a.s.cu_q + b);
   const int n = __ldg(a.s.cu_q + b + 1) - q0;
   const int L = __ldg(a.s.cu_k + b + 1) - __ldg(a.s.cu_k + b);
+  if (!(q0 <= t && t - q0 < n && n <= L)) return -1;
   const int p = L - n + (t - q0);  // absolute position of the row
   const int lp = p / a.page_size;
   int page = -1;

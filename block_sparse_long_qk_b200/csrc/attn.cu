@@ -107,8 +107,9 @@ struct UnionWalk {
 
 // Work item -> two tiles sharing one KV head (and one request). Items run heaviest-first
 // (late query blocks have the longest causal rows). `kbase` / `len`: key row of the request's
-// position 0 and its key count; `b`: the request (page-table row).
-__device__ __forceinline__ void make_tiles(const AttnArgs& a, int item, Tile* t, int& g,
+// position 0 and its key count; `b`: the request (page-table row). Returns false (both tiles
+// absent) when the prefix sums do not describe the request consistently.
+__device__ __forceinline__ bool make_tiles(const AttnArgs& a, int item, Tile* t, int& g,
                                            int& b, int& kbase, int& len) {
   // The G query heads of a KV head form ceil(G / 2) items per query block: pairs of heads, and
   // for an odd G one single head (its CTA runs one tile).
@@ -126,7 +127,7 @@ __device__ __forceinline__ void make_tiles(const AttnArgs& a, int item, Tile* t,
   kbase = qb.kbase;
   len = qb.L;
   for (int s = 0; s < 2; ++s) {
-    if (t[s].Ig < 0) {
+    if (t[s].Ig < 0 || !qb.ok) {
       t[s].r0 = t[s].r1 = 0; t[s].cnt = 0; t[s].list = a.kv_idx; t[s].I = -1; t[s].q_lo = 0;
       continue;
     }
@@ -140,6 +141,7 @@ __device__ __forceinline__ void make_tiles(const AttnArgs& a, int item, Tile* t,
     t[s].cnt = max(0, min(t[s].cnt, a.s.max_kb));
     t[s].list = a.kv_idx + row * a.s.max_kb;
   }
+  return qb.ok;
 }
 
 template <int D, int BN, bool FP8, bool PAGED>
@@ -163,7 +165,16 @@ __global__ void __launch_bounds__(384, 1)
 
   Tile tl[2];
   int g, b, kbase, len;
-  make_tiles(a, blockIdx.x, tl, g, b, kbase, len);
+  if (!make_tiles(a, blockIdx.x, tl, g, b, kbase, len) && threadIdx.x == 0)
+    record_status(a.status, kStatusBadIndex);
+  // Producer bookkeeping: the last use of each ring slot whose load was issued, so that a CTA
+  // that gives up waits (bounded) for its own bulk copies before it exits.
+  int k_issued[C::kKSt], v_issued[C::kVSt];
+  bool q_issued = false;
+#pragma unroll
+  for (int i = 0; i < C::kKSt; ++i) k_issued[i] = -1;
+#pragma unroll
+  for (int i = 0; i < C::kVSt; ++i) v_issued[i] = -1;
 
   if (threadIdx.x == 0) {
     mbar_init(&sh.q_full, 1);
@@ -200,6 +211,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < C::kNChunk; ++c)
           tma_load_3d(smem + C::kQOff + s * C::kQBytes + c * (C::kBM * 128), &tm_q, &sh.q_full,
                       c * C::kChunkEl, tl[s].h, tl[s].q_lo);
+      q_issued = true;
       UnionWalk uw;
       uw.init(tl[0], tl[1]);
       int J, bits;
@@ -243,6 +255,8 @@ __global__ void __launch_bounds__(384, 1)
               tma_load_3d(dst + c * (BN * 128) + sgi * (seg_rows * 128), tm, full,
                           c * C::kChunkEl, g, row);
           }
+          if (which == 0) k_issued[st] = use;
+          else v_issued[st] = use;
         }
         if (sh.abort_flag) break;
       }
@@ -501,6 +515,15 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+  // After a failed wait some issued load may never have been consumed: wait (bounded) until
+  // every bulk copy of this CTA has landed, so none still writes shared memory after exit.
+  if (warp == 0 && lane == 0 && sh.abort_flag) {
+    if (q_issued) mbar_wait(&sh.q_full, 0);
+    for (int i = 0; i < C::kKSt; ++i)
+      if (k_issued[i] >= 0) mbar_wait(&sh.k_full[i], k_issued[i] & 1);
+    for (int i = 0; i < C::kVSt; ++i)
+      if (v_issued[i] >= 0) mbar_wait(&sh.v_full[i], v_issued[i] & 1);
   }
 }
 

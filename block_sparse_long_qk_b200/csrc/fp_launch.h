@@ -32,6 +32,7 @@ struct PoolArgs {
   float* q_pool;           // [Hq][total_qb][d]
   float* k_pool;           // [Hkv][total_kb][d]
   __nv_bfloat16* k_split;  // optional bf16 [2][Hkv][total_kb][d] hi / lo parts of k_pool
+  uint32_t* status;        // caller's status word, or nullptr (nothing recorded)
   Seqs s;
   int Hq, Hkv, d, page_size, max_pages, num_pages;
   int q_slices;  // column slices of Q per block (the rest of gridDim.y are K slices)
@@ -44,8 +45,10 @@ struct MaskArgs {
   uint32_t* mask_bits;  // [Hq][total_qb][ceil(max_kb / 32)]
   int32_t* kv_cnt;      // [Hq][total_qb]
   int32_t* kv_idx;      // [Hq][total_qb][max_kb]
+  uint32_t* status;     // caller's status word, or nullptr (nothing recorded)
   Seqs s;
   int Hq, Hkv, d, G, NB;
+  int fault_skip_chunk;  // test hook: CTA 0 skips the B-operand TMA load of this chunk
   float log_alpha;  // -inf for alpha = 0
   float scale;
   int flags;
@@ -115,9 +118,12 @@ namespace fp {
 
 // Query block gq of a batch: request b, absolute block index I, the request's first query
 // position P0 and key count L, the query row holding absolute position P0 (qrow0), the key row
-// of position 0 (kbase) and the global KV block of the request's block 0 (kb0).
+// of position 0 (kbase) and the global KV block of the request's block 0 (kb0). `ok` is false
+// when the prefix sums of request b do not describe it consistently (see seqs_request_ok);
+// then nothing of the block may be read or written.
 struct QBlock {
   int b, I, P0, L, qrow0, kbase, kb0;
+  bool ok;
 };
 
 #ifdef __CUDACC__
@@ -130,38 +136,81 @@ __device__ __forceinline__ int seqs_find(const int32_t* cu, int batch, int x) {
   return lo;
 }
 
+// The prefix sums are caller data that the host does not read. Before a kernel derives rows
+// from the entries of request b it checks that they describe a request the buffers can hold:
+// query blocks qb0 <= g < qb1 <= total_qb (g the block being mapped), query rows q0 .. q1 - 1
+// within [0, total_q) and at least one of them, key rows k0 .. k1 - 1 within [0, total_k) and
+// at least as many as queries, ceil(L / block) KV blocks at kb0 .. kb1 - 1 within [0, total_kb)
+// and at most max_kb of them, and ceil(L / block) - floor(P0 / block) query blocks. 64-bit
+// arithmetic, so that no sum of caller values overflows.
+__device__ __forceinline__ bool seqs_request_ok(const Seqs& s, long long g, long long qb0,
+                                                long long qb1, long long q0, long long q1,
+                                                long long k0, long long k1, long long kb0,
+                                                long long kb1) {
+  const long long nq = q1 - q0, L = k1 - k0;
+  if (!(qb0 <= g && g < qb1 && qb1 <= s.total_qb)) return false;
+  if (!(q0 >= 0 && nq >= 1 && q1 <= s.total_q)) return false;
+  if (!(k0 >= 0 && L >= nq && k1 <= s.total_k)) return false;
+  const long long nkb = (L + s.block - 1) / s.block;
+  if (!(kb0 >= 0 && kb1 - kb0 == nkb && kb1 <= s.total_kb && nkb <= s.max_kb)) return false;
+  return qb1 - qb0 == nkb - (L - nq) / s.block;
+}
+
 __device__ __forceinline__ QBlock query_block(const Seqs& s, int gq) {
   QBlock r;
+  r.ok = true;
   if (s.cu_q == nullptr) {
     r.b = 0; r.P0 = 0; r.L = s.total_k; r.qrow0 = 0; r.kbase = 0; r.kb0 = 0; r.I = gq;
     return r;
   }
   r.b = seqs_find(s.cu_qb, s.batch, gq);
+  const int qb0 = __ldg(s.cu_qb + r.b), qb1 = __ldg(s.cu_qb + r.b + 1);
   r.qrow0 = __ldg(s.cu_q + r.b);
-  const int nq = __ldg(s.cu_q + r.b + 1) - r.qrow0;
+  const int q1 = __ldg(s.cu_q + r.b + 1);
   r.kbase = __ldg(s.cu_k + r.b);
-  r.L = __ldg(s.cu_k + r.b + 1) - r.kbase;
-  r.P0 = r.L - nq;
+  const int k1 = __ldg(s.cu_k + r.b + 1);
   r.kb0 = __ldg(s.cu_kb + r.b);
-  r.I = r.P0 / s.block + (gq - __ldg(s.cu_qb + r.b));
+  const int kb1 = __ldg(s.cu_kb + r.b + 1);
+  r.ok = seqs_request_ok(s, gq, qb0, qb1, r.qrow0, q1, r.kbase, k1, r.kb0, kb1);
+  if (!r.ok) {
+    r.b = 0; r.P0 = 0; r.L = 0; r.qrow0 = 0; r.kbase = 0; r.kb0 = 0; r.I = 0;
+    return r;
+  }
+  const int nq = q1 - r.qrow0;
+  r.L = k1 - r.kbase;
+  r.P0 = r.L - nq;
+  r.I = r.P0 / s.block + (gq - qb0);
   return r;
 }
 
-// KV block gk of a batch: request b, block index J, key count L, key row of position 0.
+// KV block gk of a batch: request b, block index J, key count L, key row of position 0; `ok`
+// as for QBlock (key blocks kb0 <= gk < kb1 <= total_kb, ceil(L / block) of them, key rows
+// within [0, total_k)).
 struct KBlock {
   int b, J, L, kbase;
+  bool ok;
 };
 
 __device__ __forceinline__ KBlock key_block(const Seqs& s, int gk) {
   KBlock r;
+  r.ok = true;
   if (s.cu_k == nullptr) {
     r.b = 0; r.J = gk; r.L = s.total_k; r.kbase = 0;
     return r;
   }
   r.b = seqs_find(s.cu_kb, s.batch, gk);
-  r.kbase = __ldg(s.cu_k + r.b);
-  r.L = __ldg(s.cu_k + r.b + 1) - r.kbase;
-  r.J = gk - __ldg(s.cu_kb + r.b);
+  const long long kb0 = __ldg(s.cu_kb + r.b), kb1 = __ldg(s.cu_kb + r.b + 1);
+  const long long k0 = __ldg(s.cu_k + r.b), k1 = __ldg(s.cu_k + r.b + 1);
+  const long long L = k1 - k0;
+  r.ok = kb0 <= gk && gk < kb1 && kb1 <= s.total_kb && k0 >= 0 && L >= 1 && k1 <= s.total_k &&
+         kb1 - kb0 == (L + s.block - 1) / s.block;
+  if (!r.ok) {
+    r.b = 0; r.J = 0; r.L = 0; r.kbase = 0;
+    return r;
+  }
+  r.kbase = static_cast<int>(k0);
+  r.L = static_cast<int>(L);
+  r.J = gk - static_cast<int>(kb0);
   return r;
 }
 #endif

@@ -51,6 +51,11 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
   const int g = blockIdx.y;
   const int Ig0 = blockIdx.x * a.NB;
   const int tid = threadIdx.x;
+  // A timeout recorded in the caller's status word is sticky: do nothing (decided by one read
+  // for the whole block).
+  const bool stale = tid == 0 && a.status != nullptr &&
+                     (*reinterpret_cast<volatile uint32_t*>(a.status) & kStatusTimeout);
+  if (__syncthreads_or(stale ? 1 : 0)) return;
 
   // Row bookkeeping.
   for (int r = tid; r < R; r += kMaskThreads) {
@@ -58,7 +63,7 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
     const int h = g * a.G + r % a.G;
     if (Ig < a.s.total_qb) {
       const QBlock qb = query_block(a.s, Ig);
-      row_I[r] = qb.I;     // absolute query block: keys J = 0 .. I of the request
+      row_I[r] = qb.ok ? qb.I : -2;  // absolute query block: keys J = 0 .. I of the request
       row_kb[r] = qb.kb0;  // global KV block of the request's block 0
       row_g[r] = Ig;
     } else {
@@ -82,10 +87,19 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(MaskArgs a) {
   __syncthreads();
 
   // Key-block range this CTA needs: from block 0 of its first row's request to the diagonal
-  // block of its last row.
+  // block of its last row. With prefix sums that do not describe the requests consistently a
+  // row may fall outside it (or be refused outright): the CTA then records kStatusBadIndex and
+  // touches nothing.
   const int r_last = (min(Ig0 + a.NB, a.s.total_qb) - 1 - Ig0) * a.G;
   const int Jg_lo = row_kb[0];
   const int Jg_hi = row_kb[r_last] + row_I[r_last];
+  bool bad = false;
+  for (int r = tid; r < R; r += kMaskThreads)
+    bad |= row_I[r] == -2 || (row_g[r] >= 0 && (row_kb[r] < Jg_lo || row_kb[r] + row_I[r] > Jg_hi));
+  if (__syncthreads_or(bad ? 1 : 0)) {
+    if (tid == 0) record_status(a.status, kStatusBadIndex);
+    return;
+  }
 
   // Thread -> (key column within the chunk, row group); rows rg, rg + 4, ... of the R rows.
   const int col = tid % kMaskChunk;

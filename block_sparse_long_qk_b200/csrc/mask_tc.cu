@@ -20,6 +20,12 @@
 // In the epilogue warp w reads TMEM lane quarter w % 4 (32 query rows) and column group w / 4
 // (32 key blocks): four threads share a row, combining their partial maxima once at the pass
 // boundary and their kept counts through a per-chunk prefix in shared memory.
+//
+// Failures: every wait is bounded; one that runs out records kStatusTimeout in the caller's
+// status word and the CTA stops issuing loads and MMAs (its lists are then incomplete, which
+// the status reports). A timeout already recorded in that word makes the kernel do nothing
+// (sticky until fp_check_status clears it). A CTA whose rows the prefix sums do not describe
+// consistently records kStatusBadIndex and returns before touching any buffer.
 #include <math.h>
 #include <string.h>
 
@@ -91,6 +97,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 2);
 
   const int tid = threadIdx.x, warp = tid / 32;
+  // One thread reads the word and the block decides together (another CTA may set it at any
+  // time, so separate reads could disagree and leave the barriers below unmatched).
+  const bool stale = tid == 0 && a.status != nullptr &&
+                     (*reinterpret_cast<volatile uint32_t*>(a.status) & kStatusTimeout);
+  if (__syncthreads_or(stale ? 1 : 0)) return;
   // 1-D grid over (row tile, KV head), ordered so that the late row tiles of every KV head --
   // the longest causal rows -- launch first and the short ones fill the tail.
   const int g = blockIdx.x % a.Hkv;
@@ -104,14 +115,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     row_h[tid] = g * a.G + tid % a.G;
     if (tid < rows_used && Ig < a.s.total_qb) {
       const QBlock qb = query_block(a.s, Ig);
-      row_I[tid] = qb.I;     // absolute query block: keys J = 0 .. I of the request
-      row_kb[tid] = qb.kb0;  // global KV block of the request's block 0
+      row_I[tid] = qb.ok ? qb.I : -2;  // absolute query block: keys J = 0 .. I of the request
+      row_kb[tid] = qb.kb0;            // global KV block of the request's block 0
       row_g[tid] = Ig;
     } else {
       row_I[tid] = -1;
       row_kb[tid] = 0;
       row_g[tid] = -1;
     }
+  }
+  __syncthreads();
+  // Key-block range of the CTA: block 0 of its first row's request .. the diagonal block of
+  // its last row (rows are ordered by request, then by block). Every row must lie inside it;
+  // with inconsistent prefix sums it may not, and the CTA then touches nothing.
+  const int r_last = (min(Ig0 + rows_blk, a.s.total_qb) - 1 - Ig0) * a.G;
+  const int last = row_kb[r_last] + row_I[r_last];
+  const int Jg_lo = row_kb[0];
+  const bool bad_row = tid < kTcRows && (row_I[tid] == -2 || (row_I[tid] >= 0 &&
+                       (row_kb[tid] < Jg_lo || row_kb[tid] + row_I[tid] > last)));
+  if (__syncthreads_or(bad_row ? 1 : 0)) {
+    if (tid == 0) record_status(a.status, kStatusBadIndex);
+    return;
   }
   if (tid == 0) {
     mbar_init(&done[0], 1);
@@ -160,11 +184,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Key-block range of the CTA: block 0 of its first row's request .. the diagonal block of
-  // its last row (rows are ordered by request, then by block).
-  const int r_last = (min(Ig0 + rows_blk, a.s.total_qb) - 1 - Ig0) * a.G;
-  const int last = row_kb[r_last] + row_I[r_last];
-  const int Jg_lo = row_kb[0];
   const int nch = (last - Jg_lo) / kTcKeys + 1;
   const int W = 2 * nch;  // pass 0 chunks, then pass 1 chunks
 
@@ -206,6 +225,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // of the lo plane (rows past the group's last block carry other data or zeros; their score
   // columns are never valid).
   auto tma_chunk = [&](int w, int buf) {
+    // Test hook (fp_debug_skip_mask_load): the load is never issued, so the wait for it runs
+    // out and the kernel reports FP_ERR_TIMEOUT.
+    if (w == a.fault_skip_chunk && blockIdx.x == 0) return false;
     const int row = g * a.s.total_kb + Jg_lo + (w % nch) * kTcKeys;
     const int lo_row = a.Hkv * a.s.total_kb + row;
     uint8_t* bh = smem + C::kB + (2 * buf) * C::kTile;
@@ -216,6 +238,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tma_load_2d(bh + c * C::kBoxBytes, &tm_split, &full[buf], c * 64, row);
       tma_load_2d(bl + c * C::kBoxBytes, &tm_split, &full[buf], c * 64, lo_row);
     }
+    return true;
   };
 
   constexpr uint32_t idesc = make_idesc(1, 1, 0, kTcRows, kTcKeys);
@@ -329,8 +352,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   };
 
+  // Thread 0 alone issues loads and MMAs. After a wait of its own has run out it issues
+  // nothing more (commits only, so that every barrier the other threads wait for still
+  // completes); `lost` is the buffer of a load that was issued and never arrived.
+  bool stop = false, issued = false;
+  int lost = -1, lost_parity = 0;
   if constexpr (kTma) {
-    if (tid == 0) tma_chunk(0, 0);
+    if (tid == 0) issued = tma_chunk(0, 0);
   } else {
     fetch(0);
     store(0);
@@ -343,17 +371,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (tid == 0) {
         // chunk w has landed -> its MMAs; then, once chunk w-1's MMAs are done with the
         // other buffer, start loading chunk w+1 into it.
-        const bool ok_full = mbar_wait(&full[b], (w >> 1) & 1);
+        if (!stop && !mbar_wait(&full[b], (w >> 1) & 1)) {
+          record_status(a.status, kStatusTimeout);
+          stop = true;
+          if (issued) {
+            lost = b;
+            lost_parity = (w >> 1) & 1;
+          }
+        }
         tc_fence_after();
-        if (ok_full) issue(b);
+        if (!stop) issue(b);
         else tc_commit(&done[b]);
-        if (w + 1 < W && (w == 0 || mbar_wait(&done[b ^ 1], ((w - 1) >> 1) & 1)))
-          tma_chunk(w + 1, b ^ 1);
+        if (!stop && w + 1 < W) {
+          if (w == 0 || mbar_wait(&done[b ^ 1], ((w - 1) >> 1) & 1)) {
+            issued = tma_chunk(w + 1, b ^ 1);
+          } else {
+            record_status(a.status, kStatusTimeout);
+            stop = true;
+          }
+        }
       }
     } else {
       if (tid == 0) {
         tc_fence_after();
-        issue(b);
+        if (!stop) issue(b);
+        else tc_commit(&done[b]);
       }
       if (w + 1 < W) fetch(w + 1);  // loads in flight while the MMAs of chunk w run
     }
@@ -363,6 +405,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // either way, so the block barriers below always match.
       const bool ok = mbar_wait(&done[b ^ 1], ((w - 1) >> 1) & 1);
       if (__all_sync(0xffffffffu, ok)) process(w - 1, b ^ 1);
+      else if ((tid & 31) == 0) record_status(a.status, kStatusTimeout);
     }
     if constexpr (!kTma) {
       if (w + 1 < W) store(b ^ 1);
@@ -374,6 +417,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   {
     const bool ok = mbar_wait(&done[(W - 1) & 1], ((W - 1) >> 1) & 1);
     if (__all_sync(0xffffffffu, ok)) process(W - 1, (W - 1) & 1);
+    else if ((tid & 31) == 0) record_status(a.status, kStatusTimeout);
+  }
+  // A load that was issued but never arrived may still be writing shared memory: give it one
+  // more bounded wait before the CTA exits.
+  if constexpr (kTma) {
+    if (tid == 0 && lost >= 0) mbar_wait(&full[lost], lost_parity);
   }
 
   __syncthreads();  // the last chunk's kept counts are visible

@@ -13,6 +13,15 @@
 // overwrites every pooled value it later reads, so nothing needs clearing between calls, but
 // two calls whose work overlaps on the same GPU (for instance on two streams) race on the
 // array. Each GPU has its own copy, so calls on different GPUs do not interfere.
+//
+// The array's device address is looked up once per device and kept for the life of the
+// process, so the entry must not be used on a device after cudaDeviceReset (which destroys the
+// context the address belongs to).
+//
+// The mask here always converts the pooled keys to the bf16 hi / lo tensor-core operands inside
+// the mask kernel (no k_pool_split buffer exists to load them from), and no workspace is taken:
+// the kernels still refuse inconsistent prefix sums and bound every wait, but a failure is not
+// reported through a status word.
 #include <mutex>
 
 #include "fp_common.cuh"
@@ -76,8 +85,9 @@ extern "C" int fp_pool_and_mask_noalloc(
   float* k_pool = scratch + static_cast<size_t>(Hq) * total_blocks * d;
   int rc = fp_pool_qk(q, k, dtype, q_scale, k_scale, cu_seqlens, cu_blocks, batch, total_tokens,
                       total_blocks, Hq, Hkv, d, block, k_page_table, page_size, max_pages,
-                      num_pages, q_pool, k_pool, nullptr, stream);
+                      num_pages, q_pool, k_pool, nullptr, nullptr, stream);
   if (rc != FP_OK) return rc;
   return fp_build_block_mask(q_pool, k_pool, nullptr, cu_blocks, batch, total_blocks, max_blocks,
-                             Hq, Hkv, d, alpha, scale, flags, mask_bits, kv_cnt, kv_idx, stream);
+                             Hq, Hkv, d, alpha, scale, flags, mask_bits, kv_cnt, kv_idx, nullptr,
+                             stream);
 }

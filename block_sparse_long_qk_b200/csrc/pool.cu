@@ -7,6 +7,11 @@
 //
 // Chunked prefill: query blocks hold only the request's query positions (see Seqs).
 //
+// Faults in the caller's data are never turned into out-of-range accesses: a block whose
+// request the prefix sums do not describe consistently is skipped, and a paged token whose
+// page entry is out of range counts as zeros; both record kStatusBadIndex in the caller's
+// status word (read by fp_check_status).
+//
 // HBM-bound stream: every CTA owns one (global block, tensor, 2 KB-wide column slice) and
 // its 128 threads each own 16 contiguous bytes of the token row (8 bf16 or 16 e4m3 values),
 // walking the block's tokens with 8 independent 16-byte loads in flight per thread. A warp
@@ -37,12 +42,20 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
   size_t first_row = 0;
   if (is_q) {
     const QBlock qb = query_block(a.s, gb);
+    if (!qb.ok) {
+      if (threadIdx.x == 0) record_status(a.status, kStatusBadIndex);
+      return;
+    }
     const int lo = max(qb.P0, qb.I * a.s.block);
     const int hi = min(qb.L, (qb.I + 1) * a.s.block);
     n = hi - lo;
     first_row = static_cast<size_t>(qb.qrow0) + (lo - qb.P0);
   } else {
     const KBlock kb = key_block(a.s, gb);
+    if (!kb.ok) {
+      if (threadIdx.x == 0) record_status(a.status, kStatusBadIndex);
+      return;
+    }
     b = kb.b;
     t0 = kb.J * a.s.block;
     n = min(a.s.block, kb.L - t0);
@@ -59,15 +72,21 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
 
   // Row base of token r0 of the block (r0 % 8 == 0; with page_size % 16 == 0 the 8 rows
   // r0..r0+7 lie in one page, so one page-table lookup serves them); nullptr for a paged
-  // token whose page entry is out of range.
+  // token whose page entry is out of range (recorded in the status word).
   auto group_base = [&](int r0) -> const uint8_t* {
     size_t row;
     if (paged) {
       const int tl = t0 + r0;
       const int lp = tl / a.page_size;
-      if (lp >= a.max_pages) return nullptr;
+      if (lp >= a.max_pages) {
+        record_status(a.status, kStatusBadIndex);
+        return nullptr;
+      }
       const int page = __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp);
-      if (page < 0 || page >= a.num_pages) return nullptr;
+      if (page < 0 || page >= a.num_pages) {
+        record_status(a.status, kStatusBadIndex);
+        return nullptr;
+      }
       row = static_cast<size_t>(page) * a.page_size + (tl % a.page_size);
     } else {
       row = first_row + r0;

@@ -37,6 +37,18 @@
  *    and is asynchronous. Argument errors are reported before anything is enqueued.
  *  - Return value: FP_OK (0) or a negative FP_ERR_* code; fp_last_error_string() then holds
  *    a message for the calling thread. Nothing throws across this boundary.
+ *  - Faults found on the device (an index or page-table entry out of range, prefix sums that
+ *    do not describe the batch consistently, a pipeline wait that ran out) are recorded in the
+ *    status word of the caller's `workspace` (fp_workspace_size() bytes of device memory,
+ *    256-byte aligned, zeroed once before first use) and read with fp_check_status. The
+ *    kernels never turn such a fault into an out-of-range access: the affected block is
+ *    skipped and its outputs are left unwritten or incomplete. For the pool and mask calls the
+ *    workspace may be NULL (then nothing is recorded); the attention and append calls require
+ *    it. One workspace shared by the calls of a step reports the whole step.
+ *  - Prefix sums are read on the device only. Each block a kernel maps checks the entries of
+ *    its own request: rows and blocks within the totals passed, a non-empty query range no
+ *    longer than the key range, and block counts equal to the ceil-divisions stated below (and
+ *    at most max_blocks). A violation is FP_ERR_BAD_INDEX.
  */
 #ifndef FPSPARSE_H_
 #define FPSPARSE_H_
@@ -63,8 +75,9 @@ extern "C" {
 #define FP_MASK_FP32 4   /* pooled scores in fp32 FFMA instead of the tensor cores (slower; the
                             same keep rule, a second implementation to cross-check) */
 
-/* Library version, e.g. 110 for 0.1.1 (0.1.1 adds the chunked-prefill calls, the paged K/V
- * append and FP_MASK_FP32). */
+/* Library version, e.g. 200 for 0.2.0. 0.1.1 added the chunked-prefill calls, the paged K/V
+ * append and FP_MASK_FP32; 0.2.0 gives the pool and mask calls a workspace (status word) and
+ * checks the prefix sums on the device. */
 int fp_version(void);
 
 /* Message describing the last error returned on the calling thread ("" if none). */
@@ -87,6 +100,9 @@ const char* fp_last_error_string(void);
  * k_pool_split  NULL, or bf16 [2, Hkv, total_blocks, d] (written): hi = bf16(k_pool) and
  *            lo = bf16(k_pool - hi), the operand split fp_build_block_mask feeds to the tensor
  *            cores; passing it on to fp_build_block_mask saves that call the conversion.
+ * workspace  NULL, or the status workspace: an out-of-range page entry (those tokens then
+ *            count as zeros) or an inconsistent request (its blocks are not written) records
+ *            FP_ERR_BAD_INDEX.
  * Supported: d in {64, 128}; block in {64, 128}; Hq % Hkv == 0; page_size a multiple of 16
  * that divides block. Q and K must be 16-byte aligned.
  */
@@ -94,7 +110,8 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
                const float* k_scale, const int32_t* cu_seqlens, const int32_t* cu_blocks,
                int batch, int total_tokens, int total_blocks, int Hq, int Hkv, int d,
                int block, const int32_t* k_page_table, int page_size, int max_pages,
-               int num_pages, float* q_pool, float* k_pool, void* k_pool_split, void* stream);
+               int num_pages, float* q_pool, float* k_pool, void* k_pool_split,
+               void* workspace, void* stream);
 
 /*
  * Stage 2: pooled block scores and the max-based dynamic threshold ("FlashPrefill:
@@ -119,11 +136,16 @@ int fp_pool_qk(const void* q, const void* k, int dtype, const float* q_scale,
  * kv_idx     int32 [Hq, total_blocks, max_blocks]: the kept request-local block indices in
  *            ascending order in the first kv_cnt entries (the rest is left untouched)
  * max_blocks largest per-request block count (host int)
+ * workspace  NULL, or the status workspace: a bounded wait that runs out records
+ *            FP_ERR_TIMEOUT (the lists of that call are then incomplete), inconsistent block
+ *            prefix sums FP_ERR_BAD_INDEX (those rows are not written). A timeout recorded
+ *            earlier in the workspace makes the call do nothing until fp_check_status clears it.
  */
 int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_pool_split,
                         const int32_t* cu_blocks, int batch, int total_blocks, int max_blocks,
                         int Hq, int Hkv, int d, float alpha, float scale, int flags,
-                        uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* stream);
+                        uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx, void* workspace,
+                        void* stream);
 
 /*
  * Stage 3: causal attention over the kept KV blocks only ("FlashPrefill: Instantaneous
@@ -214,8 +236,8 @@ int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void*
  * needed to place query blocks (64 or 128).
  * fp_sparse_prefill_attn_chunked: out [total_q, Hq, d] bf16 and lse [Hq, total_q] (or NULL) for
  * the queries only. K and V are contiguous [total_k, Hkv, d] (page_table NULL) or caches read
- * through page_table (same rules as fp_sparse_prefill_attn_paged). Errors as fp_pool_qk,
- * fp_build_block_mask and fp_sparse_prefill_attn respectively.
+ * through page_table (same rules as fp_sparse_prefill_attn_paged). Errors and workspaces as
+ * fp_pool_qk, fp_build_block_mask and fp_sparse_prefill_attn respectively.
  */
 int fp_pool_qk_chunked(const void* q, const void* k, int dtype, const float* q_scale,
                        const float* k_scale, const int32_t* cu_q, const int32_t* cu_qblocks,
@@ -223,7 +245,7 @@ int fp_pool_qk_chunked(const void* q, const void* k, int dtype, const float* q_s
                        int total_k, int total_qblocks, int total_kblocks, int Hq, int Hkv,
                        int d, int block, const int32_t* k_page_table, int page_size,
                        int max_pages, int num_pages, float* q_pool, float* k_pool,
-                       void* k_pool_split, void* stream);
+                       void* k_pool_split, void* workspace, void* stream);
 
 int fp_build_block_mask_chunked(const float* q_pool, const float* k_pool,
                                 const void* k_pool_split, const int32_t* cu_q,
@@ -232,7 +254,7 @@ int fp_build_block_mask_chunked(const float* q_pool, const float* k_pool,
                                 int total_kblocks, int max_kblocks, int Hq, int Hkv, int d,
                                 int block, float alpha, float scale, int flags,
                                 uint32_t* mask_bits, int32_t* kv_cnt, int32_t* kv_idx,
-                                void* stream);
+                                void* workspace, void* stream);
 
 int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, int dtype,
                                    const float* q_scale, const float* k_scale,
@@ -280,9 +302,13 @@ int fp_append_paged_kv(const void* k_new, const void* v_new, int dtype, const in
  * Limit: (Hq + Hkv) * total_blocks * d <= 8 Mi floats; larger problems return
  * FP_ERR_INVALID_ARG with a message (use the two regular calls with caller buffers). The first
  * call on each device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture. All calls share the array
- * (each call rewrites the pooled values it reads, nothing needs clearing), so calls whose work
- * overlaps on the same GPU race. No device memory is allocated by this call.
+ * device current and keeps it for the life of the process; make that first call before any
+ * stream capture, and do not call this entry on a device after cudaDeviceReset. All calls share
+ * the array (each call rewrites the pooled values it reads, nothing needs clearing), so calls
+ * whose work overlaps on the same GPU race. No device memory is allocated by this call.
+ * Differences from the two regular calls: the mask kernel converts the pooled keys to its
+ * tensor-core operands itself (there is no k_pool_split buffer to load them from), and there is
+ * no workspace, so device-side faults are contained as in the other calls but not reported.
  */
 int fp_pool_and_mask_noalloc(const void* q, const void* k, int dtype, const float* q_scale,
                              const float* k_scale, const int32_t* cu_seqlens,
@@ -303,15 +329,25 @@ int fp_pool_and_mask_noalloc(const void* q, const void* k, int dtype, const floa
  */
 int fp_debug_skip_k_load(int union_block);
 
-/* Bytes of device workspace the attention calls need (a fixed small size). */
+/*
+ * Test hook for the mask kernel's failure path (the pages have no counterpart). Makes the NEXT
+ * fp_build_block_mask / fp_build_block_mask_chunked call issued from this thread that loads its
+ * key operands by TMA (k_pool_split given) skip, in its first CTA, the load of the given chunk
+ * of 128 key blocks (chunks of the first pass first). That CTA's bounded wait runs out after
+ * about 2 s and the workspace records FP_ERR_TIMEOUT. One-shot; FP_ERR_INVALID_ARG for a
+ * negative index.
+ */
+int fp_debug_skip_mask_load(int chunk);
+
+/* Bytes of device workspace (the status word) the calls take (a fixed small size). */
 size_t fp_workspace_size(void);
 
 /*
  * Waits for `stream`, reads and clears the status word in `workspace`, and returns FP_OK,
  * FP_ERR_TIMEOUT or FP_ERR_BAD_INDEX (or FP_ERR_CUDA if the stream itself failed).
  * The workspace must have been zeroed once before its first use (e.g. cudaMemset).
- * A recorded timeout is sticky: attention launches on that workspace do no work (their CTAs
- * exit at once) until this call has cleared it.
+ * A recorded timeout is sticky: mask and attention launches on that workspace do no work
+ * (their CTAs exit at once) until this call has cleared it.
  */
 int fp_check_status(void* workspace, void* stream);
 

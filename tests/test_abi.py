@@ -101,7 +101,7 @@ def test_paged_attention_rejects_bad_paging(over, msg):
 ])
 def test_mask_error_messages(args, code, msg):
     lib = fp.library()
-    rc = lib.fp_build_block_mask(*args, 0.1, 3, None, 16, 16, None)
+    rc = lib.fp_build_block_mask(*args, 0.1, 3, None, 16, 16, None, None)
     assert rc == code
     assert msg in lib.fp_last_error_string()
 
@@ -120,6 +120,7 @@ def test_noalloc_refuses_problems_past_its_scratch():
 def test_debug_hook_and_status_reject_bad_arguments():
     lib = fp.library()
     assert lib.fp_debug_skip_k_load(-1) == -1
+    assert lib.fp_debug_skip_mask_load(-1) == -1
     assert lib.fp_check_status(None, None) == -1
     assert b"workspace" in lib.fp_last_error_string()
 
@@ -127,7 +128,7 @@ def test_debug_hook_and_status_reject_bad_arguments():
 def test_mask_rejects_alpha_out_of_range():
     lib = fp.library()
     rc = lib.fp_build_block_mask(16, 16, None, None, 1, 4, 4, 8, 2, 128, 1.5, 0.1, 3, None, 16,
-                                 16, None)
+                                 16, None, None)
     assert rc == -1
     assert b"alpha" in lib.fp_last_error_string()
 
@@ -170,13 +171,13 @@ def test_chunked_mask_and_pool_reject_bad_arguments():
     lib = fp.library()
     # mask: block size is needed to place query blocks
     rc = lib.fp_build_block_mask_chunked(16, 16, None, 16, 16, 16, 16, 2, 4, 9, 5, 8, 2, 128, 96,
-                                         0.1, 0.1, 3, None, 16, 16, None)
+                                         0.1, 0.1, 3, None, 16, 16, None, None)
     assert rc == -2
     rc = lib.fp_build_block_mask_chunked(16, 16, None, None, 16, 16, 16, 2, 4, 9, 5, 8, 2, 128,
-                                         128, 0.1, 0.1, 3, None, 16, 16, None)
+                                         128, 0.1, 0.1, 3, None, 16, 16, None, None)
     assert rc == -1
     rc = lib.fp_pool_qk_chunked(16, 16, 0, None, None, 16, 16, 16, 16, 2, 1001, 1000, 4, 9, 8, 2,
-                                128, 128, None, 0, 0, 0, 16, 16, None, None)
+                                128, 128, None, 0, 0, 0, 16, 16, None, None, None)
     assert rc == -1 and b"total_q" in lib.fp_last_error_string()
 
 
@@ -197,9 +198,9 @@ def test_empty_inputs_return_ok_without_launching():
     """No tokens: every stage returns FP_OK before any CUDA call (this runs without a GPU)."""
     lib = fp.library()
     assert lib.fp_pool_qk(16, 16, 0, None, None, None, None, 1, 0, 0, 8, 2, 128, 128, None, 0, 0,
-                          0, 16, 16, None, None) == 0
+                          0, 16, 16, None, None, None) == 0
     assert lib.fp_build_block_mask(16, 16, None, None, 1, 0, 0, 8, 2, 128, 0.1, 0.1, 3, None, 16,
-                                   16, None) == 0
+                                   16, None, None) == 0
     assert _bad_attn(T=0, tb=0, mb=0) == 0
     assert lib.fp_append_paged_kv(16, 16, 0, 16, 16, 1, 0, 2, 128, 16, 64, 1, 1, 16, 16, 256,
                                   None) == 0
@@ -213,7 +214,7 @@ def test_host_index_arrays_are_refused_before_launch():
     cb = np.array([0, 2, 3], dtype=np.int32)
     lib = fp.library()
     rc = lib.fp_pool_qk(16, 16, 0, None, None, cu.ctypes.data, cb.ctypes.data, 2, 300, 3, 8, 2,
-                        128, 128, None, 0, 0, 0, 16, 16, None, None)
+                        128, 128, None, 0, 0, 0, 16, 16, None, None, None)
     assert rc == -1
     assert b"cu_" in lib.fp_last_error_string()
 
@@ -228,3 +229,21 @@ def test_binding_refuses_cpu_tensors_views_and_mixed_dtypes():
         fp._same_dtype(q, k.to(torch.float8_e4m3fn))
     fp._same_dtype(q, k, None)
     assert fp._ptr(None) is None
+
+
+def test_pool_and_mask_refuse_a_misaligned_workspace():
+    """The pool and mask calls take the status workspace (NULL allowed); a misaligned one is
+    refused before anything is enqueued."""
+    lib = fp.library()
+    rc = lib.fp_pool_qk(16, 16, 0, None, None, None, None, 1, 256, 2, 8, 2, 128, 128, None, 0, 0,
+                        0, 16, 16, None, 128, None)
+    assert rc == -1 and b"workspace" in lib.fp_last_error_string()
+    rc = lib.fp_build_block_mask(16, 16, None, None, 1, 2, 2, 8, 2, 128, 0.1, 0.1, 3, None, 16,
+                                 16, 128, None)
+    assert rc == -1 and b"workspace" in lib.fp_last_error_string()
+    rc = lib.fp_pool_qk_chunked(16, 16, 0, None, None, 16, 16, 16, 16, 2, 300, 1000, 4, 9, 8, 2,
+                                128, 128, None, 0, 0, 0, 16, 16, None, 64, None)
+    assert rc == -1 and b"workspace" in lib.fp_last_error_string()
+    rc = lib.fp_build_block_mask_chunked(16, 16, None, 16, 16, 16, 16, 2, 4, 9, 5, 8, 2, 128, 128,
+                                         0.1, 0.1, 3, None, 16, 16, 64, None)
+    assert rc == -1 and b"workspace" in lib.fp_last_error_string()

@@ -360,7 +360,8 @@ def test_strided_views_and_host_prefix_sums_are_refused(cuda_device):
     kp = torch.empty((2, 3, 128), device=cuda_device)
     rc = fp.library().fp_pool_qk(fp._ptr(q), fp._ptr(k), 0, None, None, cu.ctypes.data,
                                  fp._ptr(b.cu_blocks), 2, 256, 3, 4, 2, 128, 128, None, 0, 0,
-                                 0, fp._ptr(qp), fp._ptr(kp), None, fp._stream(q.device))
+                                 0, fp._ptr(qp), fp._ptr(kp), None, None,
+                                 fp._stream(q.device))
     assert rc == -1 and b"host memory" in fp.library().fp_last_error_string()
     torch.cuda.synchronize()
 
