@@ -7,14 +7,18 @@ One step = the whole path over one layer's synthetic inputs: fp_pool_qk -> fp_bu
 -> fp_sparse_prefill_attn (or the paged entry), launched through the C ABI. Inputs (Q 1 GiB,
 K and V 256 MiB each at 128K) are larger than the 126 MB L2, so steps run back to back
 without an L2 flush. Timing: CUDA events on the launching stream, W warm-up steps, then K
-timed steps bracketed by barrier + synchronize; multi-GPU runs are independent replicas
-(each rank its own layer, no collective) and report the max over ranks.
+timed steps bracketed by barrier + synchronize; multi-GPU runs report the max over ranks and
+are either independent replicas (each rank its own layer; value = ms per step / N, weak
+scaling) or, with --split heads, one layer split by KV-head group (each rank the whole path on
+its heads, no exchange; value = ms per step, strong scaling). The only collectives are the
+timing barrier and the max-reduction.
 
 Prints one JSON line (rank 0).
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -239,6 +243,8 @@ def cpu_baseline(inp, rows_sample=32, seed=5):
     sample = (f"pool+mask in full ({1e3 * (t1 - t0):.0f} ms) + attention on {rows_sample} of "
               f"{total_rows} (head, query-block) rows ({1e3 * (t2 - t1):.0f} ms), "
               f"extrapolated to the layer")
+    sample += (f"; cores = the {cores} threads numpy's BLAS may use: the oracle's per-block and "
+               "per-row Python loops run on one core, only its matrix products use more")
     return {"value": round(ms, 3), "unit": "ms/layer", "cores": cores, "kind": "oracle",
             "sample": sample}
 
@@ -297,81 +303,205 @@ def _config(w, args):
                         f"{w.dtype}" + (f" paged{w.page_size}" if w.page_size else "")
                         + (f" chunked: q={sum(w.q_lens)} new tokens after cached prefixes"
                            if w.q_lens is not None else ""),
-            "tokens": w.total_tokens, "requests": w.batch, "parallelism": f"replicas{args.gpus}",
+            "tokens": w.total_tokens, "requests": w.batch,
+            "parallelism": (f"heads{args.gpus}" if args.split == "heads"
+                            else f"replicas{args.gpus}"),
             "l2": "inputs larger than L2 (no flush)"}
 
 
-def run_native(args, world, rank, local):
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    w = S.WORKLOADS[args.workload]
-    inp = S.make_inputs(args.workload, seed=S.DEFAULT_SEEDS[w.name] + 1000 * rank)
-    layer = Layer(inp, dev)
-    peaks, peak_src = _peaks()
+def shard_inputs(inp, rank, world):
+    """The part of one layer that rank ``rank`` runs when the layer is split by KV-head group
+    (``fp.head_shard``): contiguous copies of its query heads and KV heads, as the projections
+    of a tensor-parallel model would produce them, with the head counts set to the slice's."""
+    w = inp.workload
+    qs, ks = fp.head_shard(w.Hq, w.Hkv, rank, world)
 
-    for _ in range(args.warmup):
+    def cut(t, sl, dim):
+        if t is None:
+            return None
+        idx = [slice(None)] * t.dim()
+        idx[dim] = sl
+        return t[tuple(idx)].contiguous()
+    ws = dataclasses.replace(w, name=f"{w.name}/heads{world}", Hq=qs.stop - qs.start,
+                             Hkv=ks.stop - ks.start)
+    return dataclasses.replace(inp, workload=ws, q=cut(inp.q, qs, 1), k=cut(inp.k, ks, 1),
+                               v=cut(inp.v, ks, 1), q_scale=cut(inp.q_scale, qs, 0),
+                               k_scale=cut(inp.k_scale, ks, 0), v_scale=cut(inp.v_scale, ks, 0),
+                               k_cache=cut(inp.k_cache, ks, 2), v_cache=cut(inp.v_cache, ks, 2))
+
+
+def measure_e4m3_peak(dev, n=8192, reps=10):
+    """Dense e4m3 GEMM rate of this GPU in TFLOP/s: torch._scaled_mm on n^3 (fp32 accumulate,
+    bf16 out), best of ``reps`` launches timed with CUDA events -- the same kind of burst figure
+    as the bf16 peak of the measured-peaks file. None if the call is unavailable."""
+    try:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()  # column-major operand
+        one = torch.ones((), device=dev)
+
+        def mm():
+            return torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            mm()
+        best = math.inf
+        for _ in range(reps):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            mm()
+            e.record()
+            torch.cuda.synchronize(dev)
+            best = min(best, s.elapsed_time(e))
+        del a, b
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
+def time_layer(layer, steps, warmup, world, dev, local):
+    """W warm-up steps, then K steps timed with CUDA events between two barriers, with the SM
+    clocks sampled over the timed region. Returns the max-over-ranks ms per step, the per-step
+    stage times, the clock record and the last step's lists."""
+    # The clock sampler starts before the warm-up, so that starting it does not land in the
+    # timed region; its samples cover the warm-up and the timed steps.
+    clocks = Clocks(local)
+    clocks.start()
+    for _ in range(warmup):
         layer.step()
     torch.cuda.synchronize(dev)
     fp.check_status(dev)
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    clocks = Clocks(local)
-    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    # A ~25 ms device-side spin ahead of the start event lets the host enqueue the timed steps
+    # before the GPU reaches them, so a host-side stall while launching cannot leave the GPU
+    # idle inside the timed region (the events would count that idle time).
+    torch.cuda._sleep(50_000_000)
     t_start.record()
-    for i in range(args.steps):
+    for i in range(steps):
         out, cnt, idx = layer.step(evs[i])
     t_end.record()
     torch.cuda.synchronize(dev)
     barrier(world)
     clk = clocks.stop()
     fp.check_status(dev)
-    total_ms = t_start.elapsed_time(t_end)
-    ms_step = max_over_ranks(total_ms / args.steps, world, dev)
-    pool_l = [e[0].elapsed_time(e[1]) for e in evs]
-    mask_l = [e[1].elapsed_time(e[2]) for e in evs]
-    attn_l = [e[2].elapsed_time(e[3]) for e in evs]
+    ms_step = max_over_ranks(t_start.elapsed_time(t_end) / steps, world, dev)
+    stages = {"pool": [e[0].elapsed_time(e[1]) for e in evs],
+              "mask": [e[1].elapsed_time(e[2]) for e in evs],
+              "attn": [e[2].elapsed_time(e[3]) for e in evs]}
+    return ms_step, stages, clk, cnt, idx
+
+
+def roofline(w, alg, executed, attn_ms, peaks, peak_src, clk, e4m3_peak):
+    """The attention kernel's roofline entry. The denominator is the measured BURST dense rate
+    of the kernel's own input type: the kernel is timed per launch (~10 ms), not in a
+    seconds-long loop, so the sustained figure (taken at a lower clock under the power cap) is
+    reported beside it, not used. e4m3 takes the live-measured e4m3 GEMM rate, else 2x the bf16
+    burst (the datasheet ratio)."""
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained")
+    e4m3 = w.dtype == "e4m3"
+    if e4m3:
+        if e4m3_peak:
+            peak, src = e4m3_peak, "e4m3 dense GEMM (torch._scaled_mm 8192^3), measured in this run, burst"
+        else:
+            peak, src = 2.0 * burst, f"{peak_src} bf16 burst x2 (datasheet e4m3/bf16 ratio)"
+    else:
+        peak, src = burst, f"{peak_src} bf16 burst (cuBLAS 8192^3 best of 10)"
+    ach = alg / (attn_ms * 1e-3) / 1e12
+    exe = executed / (attn_ms * 1e-3) / 1e12
+    traffic = None
+    tf = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if os.path.exists(tf):
+        traffic = json.load(open(tf)).get(w.name) or None
+    nominal = NOMINAL_BF16_TFLOPS * (2.0 if e4m3 else 1.0)
+    r = {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+         "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": src,
+         "executed_tflops": round(exe, 2), "executed_frac": round(exe / peak, 4),
+         # the datasheet's dense figure, for context (2.25 PFLOP/s bf16, 4.5 e4m3)
+         "nominal_peak": nominal, "frac_of_nominal": round(ach / nominal, 4)}
+    if sustained:
+        sp = sustained * (e4m3_peak / burst if e4m3 and e4m3_peak else (2.0 if e4m3 else 1.0))
+        r["frac_of_sustained"] = round(ach / sp, 4)
+    sm, sm_max = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    if sm and sm_max:
+        # what the same cycles would deliver at the maximum SM clock (the kernel runs under the
+        # 1 kW power cap at the sampled median clock)
+        r["achieved_at_max_clock"] = round(ach * sm_max / sm, 2)
+        r["frac_at_max_clock"] = round(ach * sm_max / sm / peak, 4)
+    return r
+
+
+def measure_extra(name, args, dev, local, peaks, peak_src, e4m3_peak):
+    """Device-side figures of a second workload in the same run (the e4m3 128K layer beside
+    the bf16 one): stage times, work and roofline, timed as the main workload is."""
+    w = S.WORKLOADS[name]
+    inp = S.make_inputs(name)
+    layer = Layer(inp, dev)
+    del inp
+    ms_step, st, clk, cnt, idx = time_layer(layer, args.steps, args.warmup, 1, dev, local)
+    alg, executed, density = work_counts(w, cnt, idx)
+    attn_ms = statistics.mean(st["attn"])
+    pool_bytes, pm_bytes = pool_mask_bytes(w)
+    pm_ms = statistics.mean(st["pool"]) + statistics.mean(st["mask"])
+    out = {"workload": _config(w, args)["workload"], "ms_per_step": round(ms_step, 4),
+           "stages_ms": {k: round(statistics.mean(v), 4) for k, v in st.items()},
+           "block_density": round(density, 5),
+           "attn_tflop": {"algorithmic": round(alg / 1e12, 3), "executed": round(executed / 1e12, 3)},
+           "pool_mask_frac_hbm": round(pm_bytes / (pm_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+           "roofline": roofline(w, alg, executed, attn_ms, peaks, peak_src, clk, e4m3_peak),
+           "clocks": clk}
+    del layer
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_native(args, world, rank, local):
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = S.WORKLOADS[args.workload]
+    heads = args.split == "heads"
+    # replicas: each rank its own layer; head split: every rank the same layer, its own heads
+    inp = S.make_inputs(args.workload, seed=S.DEFAULT_SEEDS[w.name] + (0 if heads else 1000 * rank))
+    if heads:
+        inp = shard_inputs(inp, rank, world)
+        w = inp.workload
+    layer = Layer(inp, dev)
+    peaks, peak_src = _peaks()
+    per_layer = 1 if heads else world   # layers the job completes per step
+
+    ms_step, st, clk, cnt, idx = time_layer(layer, args.steps, args.warmup, world, dev, local)
+    pool_l, mask_l, attn_l = st["pool"], st["mask"], st["attn"]
     pool_ms, mask_ms, attn_ms = (statistics.mean(x) for x in (pool_l, mask_l, attn_l))
 
     alg, executed, density = work_counts(w, cnt, idx)
     pool_bytes, pm_bytes = pool_mask_bytes(w)
-    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    if w.dtype == "e4m3":
-        peak_t *= 2.0   # e4m3 dense rate = 2x bf16 (nominal ratio); no measured e4m3 peak
-    nominal_t = NOMINAL_BF16_TFLOPS * (2.0 if w.dtype == "e4m3" else 1.0)
-    traffic = None
-    tf = os.path.join(ROOT, "profiles", "attn_traffic.json")
-    if os.path.exists(tf):
-        t = json.load(open(tf)).get(w.name)
-        if t:
-            traffic = t
-    roof = {"bound": "tensor", "achieved": round(alg / (attn_ms * 1e-3) / 1e12, 2),
-            "peak": peak_t, "unit": "TFLOP/s",
-            "frac": round(alg / (attn_ms * 1e-3) / 1e12 / peak_t, 4), "traffic": traffic,
-            "peak_source": f"{peak_src} bf16 sustained" + (" x2 (e4m3 nominal ratio)"
-                                                          if w.dtype == "e4m3" else ""),
-            "executed_tflops": round(executed / (attn_ms * 1e-3) / 1e12, 2),
-            "executed_frac": round(executed / (attn_ms * 1e-3) / 1e12 / peak_t, 4),
-            # the datasheet's dense figure, for context (2.25 PFLOP/s bf16, 4.5 e4m3)
-            "nominal_peak": nominal_t,
-            "frac_of_nominal": round(alg / (attn_ms * 1e-3) / 1e12 / nominal_t, 4)}
+    extra_names = ([] if (args.no_extra or world > 1 or w.name != "llama128k")
+                   else ["fp8_128k"])
+    e4m3_peak = None
+    if w.dtype == "e4m3" or extra_names:
+        e4m3_peak = measure_e4m3_peak(dev)
+    roof = roofline(w, alg, executed, attn_ms, peaks, peak_src, clk, e4m3_peak)
 
     # e2e: host (pinned) inputs -> device, the layer, output -> host, per step
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(layer, inp, dev, args, world)
+        e2e = run_e2e(layer, inp, dev, args, world, per_layer)
+    del layer
+    torch.cuda.empty_cache()
+    extra = {n: measure_extra(n, args, dev, local, peaks, peak_src, e4m3_peak)
+             for n in extra_names}
 
     if rank == 0:
         cb = None
         if world == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline(inp, rows_sample=args.ref_rows)
         line = {
-            "metric": METRIC, "value": round(ms_step / world, 4), "unit": "ms/layer",
+            "metric": METRIC, "value": round(ms_step / per_layer, 4), "unit": "ms/layer",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
+            "ms_per_step": round(ms_step, 4), "higher_is_better": False,
+            "scaling": "strong" if heads else "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": _config(w, args),
             "stages_ms": {"pool": round(pool_ms, 4), "mask": round(mask_ms, 4),
@@ -397,10 +527,14 @@ def run_native(args, world, rank, local):
             "gpu_launches": 3 * args.steps,
             "clocks": clk,
         }
+        if e4m3_peak:
+            line["e4m3_peak_tflops_measured"] = round(e4m3_peak, 1)
+        if extra:
+            line["extra"] = extra
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(layer, inp, dev, args, world):
+def run_e2e(layer, inp, dev, args, world, per_layer):
     """Same metric through the public API with host buffers: every step copies Q, K, V (or the
     paged K/V caches) from pinned host memory, runs the whole path and copies the output back.
     ``fp.HostPipeline`` overlaps one step's copies with the neighbouring steps' kernels; the
@@ -456,7 +590,7 @@ def run_e2e(layer, inp, dev, args, world):
     fp.check_status(dev)
     h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + \
         hv.numel() * hv.element_size()
-    return {"value": round(ms / world, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
+    return {"value": round(ms / per_layer, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": houts[0].numel() * houts[0].element_size(), "steps": steps,
             "pipelined": "copy-in, kernels and copy-out of neighbouring steps overlap",
             "inputs": ("chunk Q, K, V rows (cached prefix resident in the paged cache; the "
@@ -473,6 +607,11 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: independent layers per rank (replicas, weak scaling) or one "
+                         "layer split by KV-head group (heads, strong scaling; no exchange)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the e4m3 128K layer that the default bf16 128K run also times")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     try:
