@@ -30,7 +30,7 @@ import torch
 
 __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_attn",
            "sparse_prefill_attn_paged", "sparse_prefill", "check_status", "workspace",
-           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "MASK_FP32", "header_symbols",
+           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "MASK_FP32", "OUT_PAGED", "header_symbols",
            "pool_and_mask_noalloc", "k_split_shape", "ChunkedBatch", "pool_qk_chunked",
            "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked",
            "HostPipeline", "append_paged_kv", "GraphStep", "head_shard"]
@@ -42,6 +42,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "fpsparse.h")
 FP_OK = 0
 FP_DTYPE_BF16, FP_DTYPE_E4M3 = 0, 1
 FORCE_FIRST, FORCE_DIAG, MASK_FP32 = 1, 2, 4
+OUT_PAGED = 1
 _ERRORS = {-1: "FP_ERR_INVALID_ARG", -2: "FP_ERR_UNSUPPORTED", -3: "FP_ERR_CUDA",
            -4: "FP_ERR_TIMEOUT", -5: "FP_ERR_BAD_INDEX"}
 
@@ -72,7 +73,7 @@ _SIGNATURES = {
                                 _p]),
     "fp_sparse_prefill_attn_chunked": (_i, [_p, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _i, _i,
                                             _i, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _i, _f,
-                                            _p, _p, _p, _p, _p, _p]),
+                                            _p, _p, _p, _p, _i, _p, _p]),
 }
 
 
@@ -619,10 +620,13 @@ def build_block_mask_chunked(q_pool, k_pool, cb: ChunkedBatch, alpha=0.1, *, sca
 
 def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
                                 paged: PagedKV | None = None, scale=None, q_scale=None,
-                                k_scale=None, v_scale=None, return_lse=False, out=None, ws=None):
+                                k_scale=None, v_scale=None, return_lse=False, out=None, ws=None,
+                                out_paged=False):
     """Attention of the chunk's queries over the kept KV blocks of the whole request ->
     (out bf16 [total_q, Hq, d], lse [Hq, total_q] or None). K/V are contiguous [total_k, Hkv,
-    d] (``k``, ``v``) or the caches of ``paged``."""
+    d] (``k``, ``v``) or the caches of ``paged``. With ``out_paged`` (paged K/V only) the output
+    is written in the caches' page layout instead: out [num_pages, page_size, Hq, d], the row
+    of position p of request b at slot p % page_size of page page_table[b, p // page_size]."""
     kk = paged.k_cache if paged is not None else k
     vv = paged.v_cache if paged is not None else v
     _same_dtype(q, kk, vv)
@@ -632,11 +636,14 @@ def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
     _expect_chunk_rows(cb, q, k, v, paged, need_v=True)
     _expect_lists(kv_cnt, kv_idx, Hq, cb.total_qblocks, cb.max_kblocks)
     _expect_scales(q_scale, k_scale, v_scale, Hq, Hkv)
-    _expect(out, "out", (T, Hq, d), torch.bfloat16)
+    if out_paged and paged is None:
+        raise ValueError("out_paged writes through the K/V page table: pass paged=")
+    out_shape = (paged.k_cache.shape[0], paged.page_size, Hq, d) if out_paged else (T, Hq, d)
+    _expect(out, "out", out_shape, torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
-        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty(out_shape, dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if return_lse else None
     ws = workspace(q.device) if ws is None else ws
     pt = paged.page_table if paged is not None else None
@@ -645,8 +652,8 @@ def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
         _ptr(v_scale), *cb._args(), cb.total_q, cb.total_k, cb.total_qblocks, cb.total_kblocks,
         cb.max_kblocks, Hq, Hkv, d, cb.block, _ptr(pt), paged.page_size if paged else 0,
         pt.shape[1] if pt is not None else 0, kk.shape[0] if pt is not None else 0,
-        float(scale), _ptr(kv_cnt), _ptr(kv_idx), _ptr(out), _ptr(lse), _ptr(ws),
-        _stream(q.device)))
+        float(scale), _ptr(kv_cnt), _ptr(kv_idx), _ptr(out), _ptr(lse),
+        OUT_PAGED if out_paged else 0, _ptr(ws), _stream(q.device)))
     return out, lse
 
 
@@ -672,8 +679,9 @@ def append_paged_kv(k_new, v_new, cb: ChunkedBatch, paged: PagedKV, *, ws=None):
 def sparse_prefill_chunked(q, k, v, cb: ChunkedBatch, alpha=0.1, *,
                            paged: PagedKV | None = None, scale=None, q_scale=None,
                            k_scale=None, v_scale=None, return_lse=False,
-                           flags=FORCE_FIRST | FORCE_DIAG, out=None):
-    """The whole path for a chunked batch. Returns (out, lse or None, kv_cnt, kv_idx)."""
+                           flags=FORCE_FIRST | FORCE_DIAG, out=None, out_paged=False):
+    """The whole path for a chunked batch. Returns (out, lse or None, kv_cnt, kv_idx);
+    ``out_paged`` as for ``sparse_prefill_attn_chunked``."""
     d = q.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -686,7 +694,7 @@ def sparse_prefill_chunked(q, k, v, cb: ChunkedBatch, alpha=0.1, *,
                                                  flags=flags, mask_bits=False, k_split=k_split)
     out, lse = sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb, paged=paged, scale=scale,
                                            q_scale=q_scale, k_scale=k_scale, v_scale=v_scale,
-                                           return_lse=return_lse, out=out)
+                                           return_lse=return_lse, out=out, out_paged=out_paged)
     return out, lse, kv_cnt, kv_idx
 
 

@@ -268,7 +268,7 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
               const float* k_scale, const float* v_scale, const fp::Seqs& s, int Hq, int Hkv,
               int d, const int32_t* page_table, int page_size, int max_pages, int num_pages,
               float scale, const int32_t* kv_cnt, const int32_t* kv_idx, void* out, float* lse,
-              void* workspace, void* stream) {
+              int out_flags, void* workspace, void* stream) {
   if (!q || !k || !v || !out || !kv_cnt || !kv_idx || !workspace)
     return fail(FP_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -280,6 +280,9 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
   if (rc) return rc;
   if (page_table && s.cu_k == nullptr)
     return fail(FP_ERR_INVALID_ARG, "paged attention needs the varlen prefix sums");
+  if (out_flags & ~FP_OUT_PAGED) return fail(FP_ERR_INVALID_ARG, "unknown output flags %d", out_flags);
+  if ((out_flags & FP_OUT_PAGED) && !page_table)
+    return fail(FP_ERR_INVALID_ARG, "FP_OUT_PAGED writes through the K/V page table: pass one");
   const int G = Hq / Hkv;
   fp::AttnArgs a{};
   a.kv_cnt = kv_cnt;
@@ -301,6 +304,7 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
   a.num_items = Hkv * ((G + 1) / 2) * s.total_qb;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.fault_skip_k = g_fault_skip_k;
+  a.out_paged = (out_flags & FP_OUT_PAGED) ? 1 : 0;
   g_fault_skip_k = -1;
   fp::AttnLaunch L{};
   L.q = q;
@@ -380,7 +384,7 @@ int fp_sparse_prefill_attn(const void* q, const void* k, const void* v, int dtyp
   return attn_impl(q, k, v, dtype, q_scale, k_scale, v_scale,
                    plain_seqs(cu_seqlens, cu_blocks, batch, total_tokens, total_blocks,
                               max_blocks, block),
-                   Hq, Hkv, d, nullptr, 0, 0, 0, scale, kv_cnt, kv_idx, out, lse, workspace,
+                   Hq, Hkv, d, nullptr, 0, 0, 0, scale, kv_cnt, kv_idx, out, lse, 0, workspace,
                    stream);
 }
 
@@ -404,7 +408,7 @@ int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void*
                    plain_seqs(cu_seqlens, cu_blocks, batch, total_tokens, total_blocks,
                               max_blocks, block),
                    Hq, Hkv, d, page_table, page_size, max_pages, num_pages, scale, kv_cnt,
-                   kv_idx, out, lse, workspace, stream);
+                   kv_idx, out, lse, 0, workspace, stream);
 }
 
 static fp::Seqs chunked_seqs(const int32_t* cu_q, const int32_t* cu_qblocks,
@@ -481,7 +485,7 @@ int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, 
                                    int max_kblocks, int Hq, int Hkv, int d, int block,
                                    const int32_t* page_table, int page_size, int max_pages,
                                    int num_pages, float scale, const int32_t* kv_cnt,
-                                   const int32_t* kv_idx, void* out, float* lse,
+                                   const int32_t* kv_idx, void* out, float* lse, int out_flags,
                                    void* workspace, void* stream) {
   g_err.clear();
   int rc = check_common(dtype, q_scale, k_scale, v_scale, true, cu_q, cu_qblocks, batch,
@@ -494,7 +498,7 @@ int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, 
                    chunked_seqs(cu_q, cu_qblocks, cu_k, cu_kblocks, batch, total_q, total_k,
                                 total_qblocks, total_kblocks, max_kblocks, block),
                    Hq, Hkv, d, page_table, page_size, max_pages, num_pages, scale, kv_cnt,
-                   kv_idx, out, lse, workspace, stream);
+                   kv_idx, out, lse, out_flags, workspace, stream);
 }
 
 int fp_append_paged_kv(const void* k_new, const void* v_new, int dtype, const int32_t* cu_q,

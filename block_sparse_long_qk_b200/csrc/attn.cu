@@ -357,10 +357,10 @@ __global__ void __launch_bounds__(384, 1)
     // over the S columns in TMEM; returns the row sum. Four independent partial sums keep the
     // add chain short.
     // With e4m3 inputs the MMAs run twice as fast and the MUFU ex2 unit (4 lanes per clock per
-    // SM sub-partition) becomes the limit: there, three column pairs in eight off the diagonal
-    // take the FMA-pipe polynomial instead (measured at 128K: 8.10 ms vs 8.27 with 1/4, 8.57
-    // with 1/2, 8.76 with none). With bf16 the extra FMA work costs more than it saves, so
-    // every exponential uses MUFU ex2.
+    // SM sub-partition) becomes the limit: there, two column pairs in eight off the diagonal
+    // take the FMA-pipe polynomial instead (measured at 128K, interleaved: 7.62 ms median
+    // against 8.02 with 1/8 or 3/8 and 8.27 with 1/2). With bf16 the extra FMA work costs
+    // more than it saves, so every exponential uses MUFU ex2.
     constexpr bool kPolyExp = FP8;
     auto p_pass = [&](const float* s_row, float mu, auto diag_tag) -> float {
       constexpr bool diag = decltype(diag_tag)::value;
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(384, 1)
               if (c0 + c > r) x.x = -INFINITY;
               if (c0 + c + 1 > r) x.y = -INFINITY;
             }
-            pp[c / 2] = (kPolyExp && !diag && (c / 2) % 8 >= 5)
+            pp[c / 2] = (kPolyExp && !diag && (c / 2) % 8 >= 6)
                             ? exp2_poly2(x)
                             : make_float2(ex2(x.x), ex2(x.y));
           }
@@ -471,11 +471,27 @@ __global__ void __launch_bounds__(384, 1)
     const bool fin = ok && !sh.abort_flag && mbar_wait(&sh.o_final[t], 0);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
+      // Output row of tile row r: its query row, or, with a paged output, the slot of its
+      // absolute position in the page the K/V page table gives (an entry out of range skips
+      // the row and records kStatusBadIndex).
+      bool valid = r >= T.r0 && r < T.r1;
+      size_t out_row = static_cast<size_t>(T.q_lo + r);
+      if (a.out_paged && valid) {
+        const int pos = T.I * BN + r;
+        const int lp = pos / a.page_size;
+        const int pg = lp < a.max_pages
+                           ? __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp) : -1;
+        if (pg >= 0 && pg < a.num_pages) {
+          out_row = static_cast<size_t>(pg) * a.page_size + pos % a.page_size;
+        } else {
+          record_status(a.status, kStatusBadIndex);
+          valid = false;
+        }
+      }
+      __nv_bfloat16* orow = a.out + (out_row * a.Hq + T.h) * D;
       if (n > 0) {
         float inv = (l > 0.f) ? 1.f / l : 0.f;
         if constexpr (FP8) inv *= __ldg(a.v_scale + g);
-        const bool valid = r >= T.r0 && r < T.r1;
-        __nv_bfloat16* orow = a.out + (static_cast<size_t>(T.q_lo + r) * a.Hq + T.h) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           float o[32];
@@ -496,9 +512,8 @@ __global__ void __launch_bounds__(384, 1)
         if (valid && a.lse != nullptr)
           a.lse[static_cast<size_t>(T.h) * a.s.total_q + T.q_lo + r] =
               (l > 0.f) ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
-      } else if (r >= T.r0 && r < T.r1) {
+      } else if (valid) {
         // No kept block at all: the row attends to nothing; write zeros / -inf.
-        __nv_bfloat16* orow = a.out + (static_cast<size_t>(T.q_lo + r) * a.Hq + T.h) * D;
         for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         if (a.lse != nullptr)
           a.lse[static_cast<size_t>(T.h) * a.s.total_q + T.q_lo + r] = -INFINITY;

@@ -70,6 +70,7 @@ struct AttnArgs {
   int G;                               // query heads per KV head
   int num_items;                        // Hkv * ceil(G / 2) * total_qb
   int fault_skip_k;                     // test hook: CTA 0 skips the K load of this union block
+  int out_paged;                        // out is [num_pages, page_size, Hq, d] via page_table
   float scale_log2;                     // softmax scale * log2(e)
 };
 

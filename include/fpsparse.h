@@ -75,6 +75,9 @@ extern "C" {
 #define FP_MASK_FP32 4   /* pooled scores in fp32 FFMA instead of the tensor cores (slower; the
                             same keep rule, a second implementation to cross-check) */
 
+#define FP_OUT_PAGED 1   /* out_flags of fp_sparse_prefill_attn_chunked: write O in the paged
+                            layout of the K/V cache (see there) */
+
 /* Library version, e.g. 200 for 0.2.0. 0.1.1 added the chunked-prefill calls, the paged K/V
  * append and FP_MASK_FP32; 0.2.0 gives the pool and mask calls a workspace (status word) and
  * checks the prefix sums on the device. */
@@ -236,8 +239,15 @@ int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void*
  * needed to place query blocks (64 or 128).
  * fp_sparse_prefill_attn_chunked: out [total_q, Hq, d] bf16 and lse [Hq, total_q] (or NULL) for
  * the queries only. K and V are contiguous [total_k, Hkv, d] (page_table NULL) or caches read
- * through page_table (same rules as fp_sparse_prefill_attn_paged). Errors and workspaces as
- * fp_pool_qk, fp_build_block_mask and fp_sparse_prefill_attn respectively.
+ * through page_table (same rules as fp_sparse_prefill_attn_paged). out_flags is 0 or
+ * FP_OUT_PAGED: then out is instead a bf16 buffer [num_pages, page_size, Hq, d] in the page
+ * layout of the K/V caches, and the output row of the query at absolute position p of request
+ * b goes to slot p % page_size of page page_table[b * max_pages + p / page_size] (the page
+ * table must be given; an entry out of range skips the row and records FP_ERR_BAD_INDEX; slots
+ * that hold no new query are not written). The epilogue thus writes O where an engine keeping
+ * per-token state in its KV page layout expects it, with no gather afterwards. lse stays
+ * [Hq, total_q]. Errors and workspaces as fp_pool_qk, fp_build_block_mask and
+ * fp_sparse_prefill_attn respectively.
  */
 int fp_pool_qk_chunked(const void* q, const void* k, int dtype, const float* q_scale,
                        const float* k_scale, const int32_t* cu_q, const int32_t* cu_qblocks,
@@ -265,7 +275,7 @@ int fp_sparse_prefill_attn_chunked(const void* q, const void* k, const void* v, 
                                    int max_kblocks, int Hq, int Hkv, int d, int block,
                                    const int32_t* page_table, int page_size, int max_pages,
                                    int num_pages, float scale, const int32_t* kv_cnt,
-                                   const int32_t* kv_idx, void* out, float* lse,
+                                   const int32_t* kv_idx, void* out, float* lse, int out_flags,
                                    void* workspace, void* stream);
 
 /*

@@ -146,8 +146,8 @@ def _bad_chunked_attn(**over):
     """A well-formed chunked attention call with fake pointers (host validation only)."""
     a = dict(q=16, k=16, v=16, dtype=0, qs=None, ks=None, vs=None, cq=16, cqb=16, ck=16, ckb=16,
              batch=2, Tq=300, Tk=1000, tqb=4, tkb=9, mkb=5, Hq=8, Hkv=2, d=128, block=128,
-             pt=None, ps=0, mp=0, npg=0, scale=0.1, cnt=16, idx=16, out=16, lse=None, ws=256,
-             stream=None)
+             pt=None, ps=0, mp=0, npg=0, scale=0.1, cnt=16, idx=16, out=16, lse=None, of=0,
+             ws=256, stream=None)
     a.update(over)
     return fp.library().fp_sparse_prefill_attn_chunked(*a.values())
 
@@ -161,6 +161,8 @@ def _bad_chunked_attn(**over):
     (dict(block=96), -2),
     (dict(pt=16, ps=48), -1),        # page size not dividing the block
     (dict(dtype=1, qs=16, ks=16, vs=16, d=64), -2),   # e4m3 needs d = 128
+    (dict(of=1), -1),                # paged output without a page table
+    (dict(of=2), -1),                # unknown output flag
 ])
 def test_chunked_attention_rejects_bad_arguments(over, code):
     assert _bad_chunked_attn(**over) == code

@@ -233,3 +233,46 @@ def test_append_reports_a_bad_page_entry(cuda_device):
     assert e.value.code == -5
     # rows whose page is valid were written (with the values they already had)
     assert torch.equal(full.k_cache, before)
+
+
+@pytest.mark.parametrize("name", ["paged", "fp8_paged"])
+def test_paged_output_layout_equals_the_contiguous_output(name, cuda_device):
+    """FP_OUT_PAGED: the attention epilogue writes each new query's output row into the K/V
+    caches' page layout (slot p % page_size of page page_table[b, p // page_size]). Gathered
+    back through the page table on the host, it equals the contiguous output bit for bit,
+    slots that hold no new query stay as they were, and lse is unchanged."""
+    if name == "fp8_paged":
+        w = dataclasses.replace(BASE, page_size=64, dtype="e4m3")
+        inp = S.make_inputs(w, seed=13, seqlens=(1100, 600, 257), q_lens=(450, 600, 64))
+    else:
+        inp, _ = _inputs(name)
+    w = inp.workload
+    q, _, _, sc = device_inputs(inp, cuda_device)
+    cb = _cb(inp, cuda_device)
+    paged = _paged(inp, cuda_device)
+    kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"])
+    qp, kp = fp.pool_qk_chunked(q, None, cb, q_scale=sc["q_scale"], k_scale=sc["k_scale"],
+                                paged=paged)
+    _, cnt, idx = fp.build_block_mask_chunked(qp, kp, cb, 0.5, mask_bits=False)
+    out, lse = fp.sparse_prefill_attn_chunked(q, None, None, cnt, idx, cb, paged=paged,
+                                              return_lse=True, **kw)
+    pages = torch.full((paged.k_cache.shape[0], paged.page_size, w.Hq, w.d), 5.0,
+                       dtype=torch.bfloat16, device=cuda_device)
+    out_p, lse_p = fp.sparse_prefill_attn_chunked(q, None, None, cnt, idx, cb, paged=paged,
+                                                  return_lse=True, out=pages, out_paged=True,
+                                                  **kw)
+    fp.check_status(cuda_device)
+    assert out_p.data_ptr() == pages.data_ptr()
+    assert torch.equal(lse_p, lse)
+    pt = inp.page_table
+    ps = paged.page_size
+    written = torch.zeros(pages.shape[:2], dtype=torch.bool)
+    cu_q = inp.cu_q.tolist()
+    for b, (n, L) in enumerate(zip(w.q_lens, w.seqlens)):
+        pos = torch.arange(L - n, L)
+        slots = pt[b, pos // ps].long() * ps + pos % ps
+        got = pages.view(-1, w.Hq, w.d)[slots.to(cuda_device)]
+        assert torch.equal(got, out[cu_q[b]:cu_q[b + 1]])
+        written.view(-1)[slots] = True
+    rest = pages.view(-1, w.Hq, w.d)[~written.view(-1).to(cuda_device)]
+    assert bool((rest == 5.0).all())
