@@ -385,3 +385,28 @@ def test_fp32_mask_matches_oracle_and_tensor_core_mask(name, cuda_device):
     for r, (x, y, ratio) in enumerate(zip(g32, gtc, run.ratios)):
         near = np.abs(ratio - alpha) <= 1e-3 * alpha
         assert not ((x != y) & ~near).any()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_split_equals_whole_layer(world, cuda_device):
+    """The multi-GPU head split (each rank the whole path on its KV-head groups, no exchange),
+    run here slice after slice on one GPU: the slices' masks and outputs, put side by side,
+    are the whole layer's bit for bit (every stage works per head, and a slice holds whole GQA
+    groups, so the attention CTAs pair the same heads)."""
+    import bench
+    w = dataclasses.replace(W["llama128k"], Hq=16, Hkv=4)
+    inp = S.make_inputs(w, seed=29, seqlens=(3000, 1700))
+    dev = cuda_device
+    b = _batch(inp, dev)
+    q, k, v, _ = device_inputs(inp, dev)
+    out, _, cnt, idx = fp.sparse_prefill(q, k, v, w.alpha, w.block, batch=b)
+    outs, cnts = [], []
+    for r in range(world):
+        part = bench.shard_inputs(inp, r, world)
+        pq, pk, pv, _ = device_inputs(part, dev)
+        o, _, c, _ = fp.sparse_prefill(pq, pk, pv, w.alpha, w.block, batch=b)
+        outs.append(o)
+        cnts.append(c)
+    fp.check_status(dev)
+    assert torch.equal(torch.cat(outs, dim=1), out)
+    assert torch.equal(torch.cat(cnts, dim=0), cnt)
