@@ -205,3 +205,27 @@ def test_append_refuses_more_new_rows_than_keys(cuda_device):
         row = kc.view(-1, 2, 128)[slot]
         assert torch.equal(row, k_new[r])
     assert int((vc.view(-1, 2, 128).float().abs().sum(dim=(1, 2)) > 0).sum()) == 100
+
+
+def test_mask_timeout_stops_the_attention_of_the_same_step(cuda_device):
+    """A step's calls share one workspace: after the mask kernel's wait ran out, its lists are
+    incomplete, and the attention launch that follows on the same workspace does no work (its
+    output buffer stays as it was) until fp_check_status reports the timeout and clears it."""
+    dev = cuda_device
+    inp = _inputs((640,), 49)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    b = fp.Batch.make((640,), 128, dev)
+    good, _, _, _ = fp.sparse_prefill(q, k, v, 0.5, 128, batch=b)
+    assert _status(dev) == 0
+    split = torch.empty(fp.k_split_shape(2, b.total_blocks, 128), dtype=torch.bfloat16,
+                        device=dev)
+    qp, kp = fp.pool_qk(q, k, 128, batch=b, k_split_out=split)
+    assert fp.library().fp_debug_skip_mask_load(0) == 0
+    _, cnt, idx = fp.build_block_mask(qp, kp, 0.5, block=128, batch=b, k_split=split)
+    out = torch.full_like(good, 7.0)
+    fp.sparse_prefill_attn(q, k, v, cnt, idx, 128, batch=b, out=out)
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())
+    assert _status(dev) == -4
+    again, _, _, _ = fp.sparse_prefill(q, k, v, 0.5, 128, batch=b)
+    assert _status(dev) == 0 and torch.equal(again, good)
