@@ -144,7 +144,9 @@ __device__ __forceinline__ bool make_tiles(const AttnArgs& a, int item, Tile* t,
   return qb.ok;
 }
 
-template <int D, int BN, bool FP8, bool PAGED>
+// OUTP: the output goes through the K/V page table (FP_OUT_PAGED; paged K/V only). A template
+// parameter, so that the other instantiations keep no page-table state live through the loop.
+template <int D, int BN, bool FP8, bool PAGED, bool OUTP>
 __global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
@@ -476,7 +478,7 @@ __global__ void __launch_bounds__(384, 1)
       // the row and records kStatusBadIndex).
       bool valid = r >= T.r0 && r < T.r1;
       size_t out_row = static_cast<size_t>(T.q_lo + r);
-      if (a.out_paged && valid) {
+      if (OUTP && valid) {
         const int pos = T.I * BN + r;
         const int lp = pos / a.page_size;
         const int pg = lp < a.max_pages
@@ -562,7 +564,7 @@ static bool make_map(CUtensorMap* m, const void* base, bool e4m3, int d, int hea
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, bool FP8, bool PAGED>
+template <int D, int BN, bool FP8, bool PAGED, bool OUTP = false>
 static cudaError_t launch_t(const AttnArgs& a, const AttnLaunch& L, cudaStream_t stream) {
   using C = AttnCfg<D, BN, FP8>;
   CUtensorMap mq, mk, mv;
@@ -570,7 +572,7 @@ static cudaError_t launch_t(const AttnArgs& a, const AttnLaunch& L, cudaStream_t
       !make_map(&mk, L.k, FP8, D, a.Hkv, L.kv_rows, L.seg_rows) ||
       !make_map(&mv, L.v, FP8, D, a.Hkv, L.kv_rows, L.seg_rows))
     return cudaErrorInvalidValue;
-  auto kern = attn_kernel<D, BN, FP8, PAGED>;
+  auto kern = attn_kernel<D, BN, FP8, PAGED, OUTP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -579,24 +581,32 @@ static cudaError_t launch_t(const AttnArgs& a, const AttnLaunch& L, cudaStream_t
   return cudaGetLastError();
 }
 
+// Paged K/V: with the paged output layout or without it.
+template <int D, int BN, bool FP8>
+static cudaError_t launch_paged(const AttnArgs& a, const AttnLaunch& L, cudaStream_t stream) {
+  return a.out_paged ? launch_t<D, BN, FP8, true, true>(a, L, stream)
+                     : launch_t<D, BN, FP8, true, false>(a, L, stream);
+}
+
 cudaError_t launch_attn(const AttnArgs& a, const AttnLaunch& L, int block, cudaStream_t stream) {
+  if (a.out_paged && !L.paged) return cudaErrorInvalidValue;
   if (L.e4m3) {
     if (L.d == 128 && block == 128)
-      return L.paged ? launch_t<128, 128, true, true>(a, L, stream)
+      return L.paged ? launch_paged<128, 128, true>(a, L, stream)
                      : launch_t<128, 128, true, false>(a, L, stream);
     return cudaErrorNotSupported;
   }
   if (L.d == 128 && block == 128)
-    return L.paged ? launch_t<128, 128, false, true>(a, L, stream)
+    return L.paged ? launch_paged<128, 128, false>(a, L, stream)
                    : launch_t<128, 128, false, false>(a, L, stream);
   if (L.d == 64 && block == 64)
-    return L.paged ? launch_t<64, 64, false, true>(a, L, stream)
+    return L.paged ? launch_paged<64, 64, false>(a, L, stream)
                    : launch_t<64, 64, false, false>(a, L, stream);
   if (L.d == 128 && block == 64)
-    return L.paged ? launch_t<128, 64, false, true>(a, L, stream)
+    return L.paged ? launch_paged<128, 64, false>(a, L, stream)
                    : launch_t<128, 64, false, false>(a, L, stream);
   if (L.d == 64 && block == 128)
-    return L.paged ? launch_t<64, 128, false, true>(a, L, stream)
+    return L.paged ? launch_paged<64, 128, false>(a, L, stream)
                    : launch_t<64, 128, false, false>(a, L, stream);
   return cudaErrorNotSupported;
 }
