@@ -70,8 +70,9 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
 #pragma unroll
   for (int i = 0; i < EPT; ++i) acc[i] = 0.f;
 
-  // Row base of token r0 of the block (r0 % 8 == 0; with page_size % 16 == 0 the 8 rows
-  // r0..r0+7 lie in one page, so one page-table lookup serves them); nullptr for a paged
+  // Row base of token r0 of the block (r0 a multiple of the group size, 8 or 16; with page_size
+  // % 16 == 0 the group's rows lie in one page, so one page-table lookup serves them); nullptr
+  // for a paged
   // token whose page entry is out of range (recorded in the status word).
   auto group_base = [&](int r0) -> const uint8_t* {
     size_t row;
@@ -120,13 +121,17 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
   };
 
   int r = 0;
-  for (; r + 8 <= n; r += 8) {
+  // Rows per group = 16-byte loads in flight per thread. An e4m3 load carries twice the values
+  // of a bf16 one, so its decode takes twice as long per byte; with 16 rows in flight the e4m3
+  // stream reaches 6.0 TB/s instead of 5.0 with 8 (128K, interleaved A/B, identical results).
+  constexpr int kInFlight = E4M3 ? 16 : 8;
+  for (; r + kInFlight <= n; r += kInFlight) {
     const uint8_t* gbase = group_base(r);
-    int4 v[8];
+    int4 v[kInFlight];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = load(gbase, u);
+    for (int u = 0; u < kInFlight; ++u) v[u] = load(gbase, u);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) accumulate(v[u]);
+    for (int u = 0; u < kInFlight; ++u) accumulate(v[u]);
   }
   if (r < n) {
     const uint8_t* gbase = group_base(r);
