@@ -30,7 +30,7 @@ import torch
 
 __all__ = ["Batch", "PagedKV", "pool_qk", "build_block_mask", "sparse_prefill_attn",
            "sparse_prefill_attn_paged", "sparse_prefill", "check_status", "workspace",
-           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "MASK_FP32", "OUT_PAGED", "header_symbols",
+           "library", "FpError", "FORCE_FIRST", "FORCE_DIAG", "MASK_FP32", "OUT_PAGED", "PAIR_QBLOCKS", "header_symbols",
            "pool_and_mask_noalloc", "k_split_shape", "ChunkedBatch", "pool_qk_chunked",
            "build_block_mask_chunked", "sparse_prefill_attn_chunked", "sparse_prefill_chunked",
            "HostPipeline", "append_paged_kv", "GraphStep", "head_shard"]
@@ -42,7 +42,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "fpsparse.h")
 FP_OK = 0
 FP_DTYPE_BF16, FP_DTYPE_E4M3 = 0, 1
 FORCE_FIRST, FORCE_DIAG, MASK_FP32 = 1, 2, 4
-OUT_PAGED = 1
+OUT_PAGED, PAIR_QBLOCKS = 1, 2
 _ERRORS = {-1: "FP_ERR_INVALID_ARG", -2: "FP_ERR_UNSUPPORTED", -3: "FP_ERR_CUDA",
            -4: "FP_ERR_TIMEOUT", -5: "FP_ERR_BAD_INDEX"}
 
@@ -621,12 +621,14 @@ def build_block_mask_chunked(q_pool, k_pool, cb: ChunkedBatch, alpha=0.1, *, sca
 def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
                                 paged: PagedKV | None = None, scale=None, q_scale=None,
                                 k_scale=None, v_scale=None, return_lse=False, out=None, ws=None,
-                                out_paged=False):
+                                out_paged=False, pair_qblocks=False):
     """Attention of the chunk's queries over the kept KV blocks of the whole request ->
     (out bf16 [total_q, Hq, d], lse [Hq, total_q] or None). K/V are contiguous [total_k, Hkv,
     d] (``k``, ``v``) or the caches of ``paged``. With ``out_paged`` (paged K/V only) the output
     is written in the caches' page layout instead: out [num_pages, page_size, Hq, d], the row
-    of position p of request b at slot p % page_size of page page_table[b, p // page_size]."""
+    of position p of request b at slot p % page_size of page page_table[b, p // page_size].
+    ``pair_qblocks`` runs every CTA on two neighbouring query blocks of one head instead of two
+    heads of a GQA group (the same output, bit for bit)."""
     kk = paged.k_cache if paged is not None else k
     vv = paged.v_cache if paged is not None else v
     _same_dtype(q, kk, vv)
@@ -653,7 +655,8 @@ def sparse_prefill_attn_chunked(q, k, v, kv_cnt, kv_idx, cb: ChunkedBatch, *,
         cb.max_kblocks, Hq, Hkv, d, cb.block, _ptr(pt), paged.page_size if paged else 0,
         pt.shape[1] if pt is not None else 0, kk.shape[0] if pt is not None else 0,
         float(scale), _ptr(kv_cnt), _ptr(kv_idx), _ptr(out), _ptr(lse),
-        OUT_PAGED if out_paged else 0, _ptr(ws), _stream(q.device)))
+        (OUT_PAGED if out_paged else 0) | (PAIR_QBLOCKS if pair_qblocks else 0), _ptr(ws),
+        _stream(q.device)))
     return out, lse
 
 

@@ -125,7 +125,7 @@ int set_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int fp_version(void) { return 200; }
+int fp_version(void) { return 300; }
 
 const char* fp_last_error_string(void) { return g_err.c_str(); }
 
@@ -280,7 +280,8 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
   if (rc) return rc;
   if (page_table && s.cu_k == nullptr)
     return fail(FP_ERR_INVALID_ARG, "paged attention needs the varlen prefix sums");
-  if (out_flags & ~FP_OUT_PAGED) return fail(FP_ERR_INVALID_ARG, "unknown output flags %d", out_flags);
+  if (out_flags & ~(FP_OUT_PAGED | FP_PAIR_QBLOCKS))
+    return fail(FP_ERR_INVALID_ARG, "unknown flags %d", out_flags);
   if ((out_flags & FP_OUT_PAGED) && !page_table)
     return fail(FP_ERR_INVALID_ARG, "FP_OUT_PAGED writes through the K/V page table: pass one");
   const int G = Hq / Hkv;
@@ -301,7 +302,20 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
   a.max_pages = max_pages;
   a.num_pages = num_pages;
   a.G = G;
-  a.num_items = Hkv * ((G + 1) / 2) * s.total_qb;
+  // Two heads of a GQA group per CTA; a head left over (odd G, all heads for G = 1, or every
+  // head with FP_PAIR_QBLOCKS) pairs two neighbouring query blocks instead. Per level of two
+  // query blocks: Hkv * head_pairs items at each block and Hkv * qpair_heads items over both;
+  // for an odd total_qb the last level has no second block and its head pairs are not launched.
+  a.head_pairs = (out_flags & FP_PAIR_QBLOCKS) ? 0 : G / 2;
+  a.qpair_heads = G - 2 * a.head_pairs;
+  {
+    const long long levels = (static_cast<long long>(s.total_qb) + 1) / 2;
+    const long long per_level = static_cast<long long>(Hkv) * (2 * a.head_pairs + a.qpair_heads);
+    const long long items =
+        levels * per_level - ((s.total_qb & 1) ? static_cast<long long>(Hkv) * a.head_pairs : 0);
+    if (items > INT_MAX) return fail(FP_ERR_INVALID_ARG, "too many attention work items");
+    a.num_items = static_cast<int>(items);
+  }
   a.scale_log2 = scale * 1.4426950408889634f;
   a.fault_skip_k = g_fault_skip_k;
   a.out_paged = (out_flags & FP_OUT_PAGED) ? 1 : 0;

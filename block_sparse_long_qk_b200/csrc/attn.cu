@@ -7,7 +7,9 @@
 // Long-Context LLM Serving", Abstract: query heads that share a KV head are packed onto the
 // same K/V loads (PackGQA), FP8 inputs, paged KV cache and continuous batching.
 //
-// B200 design (one CTA = two 128-row query tiles that read the same KV head):
+// B200 design (one CTA = two 128-row query tiles that read the same KV head: two heads of a
+// GQA group at one query block, or one head at two neighbouring query blocks; see the work
+// items below):
 //   warp 0      TMA producer: both Q tiles once, then K and V tiles of the union of the two
 //               tiles' kept-block lists into a 2-deep K ring and a 2-deep V ring.
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer. Per union block it issues
@@ -64,6 +66,13 @@ struct Tile {
   const int32_t* list;
 };
 
+// A tile's request, for the work split whose two tiles may lie in different requests: b
+// (page-table row), kbase (key row of position 0), len (key count), kb0 (its first KV block in
+// the prefix sums; kb0 + J orders the blocks of both tiles in one walk).
+struct Req {
+  int b, kbase, len, kb0;
+};
+
 struct Shared {  // placed at kBarOff
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];  // ring slots (kKSt, kVSt <= 4)
@@ -87,32 +96,39 @@ __device__ __forceinline__ int next_valid(const int32_t* list, int cnt, int& i, 
 }
 
 // Walks the ascending union of two kept-block lists; `bits` says which tiles kept the block.
+// With KEYED, the lists are merged on kb0 + J (the tiles' requests may differ: a block both
+// tiles kept, same request and same J, comes once with bits = 3; tiles of different requests
+// share none).
+template <bool KEYED>
 struct UnionWalk {
   const int32_t *l0, *l1;
-  int c0, c1, i0, i1, I0, I1, a, b;
-  __device__ void init(const Tile& t0, const Tile& t1) {
+  int c0, c1, i0, i1, I0, I1, a, b, o0, o1;
+  __device__ void init(const Tile& t0, const Tile& t1, int off0 = 0, int off1 = 0) {
     l0 = t0.list; l1 = t1.list; c0 = t0.cnt; c1 = t1.cnt; I0 = t0.I; I1 = t1.I;
+    o0 = KEYED ? off0 : 0; o1 = KEYED ? off1 : 0;
     i0 = i1 = 0;
     a = next_valid(l0, c0, i0, I0, nullptr, false);
     b = next_valid(l1, c1, i1, I1, nullptr, false);
   }
   __device__ bool next(int& J, int& bits) {
     if (a < 0 && b < 0) return false;
-    if (b < 0 || (a >= 0 && a < b)) { J = a; bits = 1; a = next_valid(l0, c0, i0, I0, nullptr, false); }
-    else if (a < 0 || b < a) { J = b; bits = 2; b = next_valid(l1, c1, i1, I1, nullptr, false); }
+    const int ka = KEYED ? a + o0 : a, kb = KEYED ? b + o1 : b;
+    if (b < 0 || (a >= 0 && ka < kb)) { J = a; bits = 1; a = next_valid(l0, c0, i0, I0, nullptr, false); }
+    else if (a < 0 || kb < ka) { J = b; bits = 2; b = next_valid(l1, c1, i1, I1, nullptr, false); }
     else { J = a; bits = 3; a = next_valid(l0, c0, i0, I0, nullptr, false); b = next_valid(l1, c1, i1, I1, nullptr, false); }
     return true;
   }
 };
 
-// Work item -> two tiles sharing one KV head (and one request). Items run heaviest-first
-// (late query blocks have the longest causal rows). `kbase` / `len`: key row of the request's
-// position 0 and its key count; `b`: the request (page-table row). Returns false (both tiles
-// absent) when the prefix sums do not describe the request consistently.
+// Head-pair split (G even): work item -> two heads of a GQA group at one query block, one
+// request. Items run heaviest-first (late query blocks have the longest causal rows). `kbase`
+// / `len`: key row of the request's position 0 and its key count; `b`: the request (page-table
+// row). Returns false (both tiles absent) when the prefix sums do not describe the request
+// consistently.
 __device__ __forceinline__ bool make_tiles(const AttnArgs& a, int item, Tile* t, int& g,
                                            int& b, int& kbase, int& len) {
-  // The G query heads of a KV head form ceil(G / 2) items per query block: pairs of heads, and
-  // for an odd G one single head (its CTA runs one tile).
+  // The G query heads of a KV head form G / 2 items per query block, pairs of heads (the
+  // general split below takes odd G; for it, this mapping would leave the last head alone).
   const int npair = (a.G + 1) / 2;
   const int per_block = a.Hkv * npair;
   const int Ig = a.s.total_qb - 1 - item / per_block;
@@ -144,9 +160,72 @@ __device__ __forceinline__ bool make_tiles(const AttnArgs& a, int item, Tile* t,
   return qb.ok;
 }
 
+// General split: work item -> two tiles that read the same KV head. Two heads of a GQA group share a query
+// block (a head pair); a head that pairing leaves over (odd G, every head when G = 1, or every
+// head when query-block pairing is forced) is paired with itself over two neighbouring query
+// blocks (the QUILT page's cross-query reuse: both tiles read every block they both kept once).
+// Items run heaviest-first in levels of two query blocks, Ig0 = total_qb - 1 - 2 * level and
+// Ig1 = Ig0 - 1: per level Hkv * hp head pairs at Ig0, Hkv * nqh query-block pairs, then
+// Hkv * hp head pairs at Ig1 (absent at the last level when total_qb is odd, so the host
+// launches none of them). Returns false (tiles absent) when the prefix sums do not describe a
+// tile's request consistently.
+__device__ __forceinline__ bool make_tiles_qp(const AttnArgs& a, int item, Tile* t, Req* rq,
+                                              int& g) {
+  const int hp = a.head_pairs, nqh = a.qpair_heads;
+  const int nA = a.Hkv * hp, nB = a.Hkv * nqh;
+  const int level = item / (2 * nA + nB);
+  int rem = item % (2 * nA + nB);
+  const int Ig0 = a.s.total_qb - 1 - 2 * level;
+  int Igs[2];
+  if (rem < nA || rem >= nA + nB) {
+    const bool second = rem >= nA;
+    if (second) rem -= nA + nB;
+    g = rem / hp;
+    t[0].h = g * a.G + 2 * (rem % hp);
+    t[1].h = t[0].h + 1;
+    Igs[0] = Igs[1] = second ? Ig0 - 1 : Ig0;
+  } else {
+    rem -= nA;
+    g = rem / nqh;
+    t[0].h = t[1].h = g * a.G + 2 * hp + rem % nqh;
+    Igs[0] = Ig0;
+    Igs[1] = Ig0 - 1;
+  }
+  bool ok = true;
+  QBlock qb{};
+  for (int s = 0; s < 2; ++s) {
+    t[s].Ig = Igs[s];
+    if (Igs[s] < 0) {
+      t[s].r0 = t[s].r1 = 0; t[s].cnt = 0; t[s].list = a.kv_idx; t[s].I = -1; t[s].q_lo = 0;
+      rq[s] = Req{0, 0, 0, 0};
+      continue;
+    }
+    if (s == 0 || Igs[1] != Igs[0]) qb = query_block(a.s, Igs[s]);
+    if (!qb.ok) {
+      ok = false;
+      t[s].r0 = t[s].r1 = 0; t[s].cnt = 0; t[s].list = a.kv_idx; t[s].I = -1; t[s].q_lo = 0;
+      rq[s] = Req{0, 0, 0, 0};
+      continue;
+    }
+    const int B = a.s.block;
+    rq[s] = Req{qb.b, qb.kbase, qb.L, qb.kb0};
+    t[s].I = qb.I;
+    t[s].q_lo = qb.qrow0 + qb.I * B - qb.P0;
+    t[s].r0 = max(0, qb.P0 - qb.I * B);
+    t[s].r1 = min(B, qb.L - qb.I * B);
+    const size_t row = static_cast<size_t>(t[s].h) * a.s.total_qb + t[s].Ig;
+    t[s].cnt = __ldg(a.kv_cnt + row);
+    t[s].cnt = max(0, min(t[s].cnt, a.s.max_kb));
+    t[s].list = a.kv_idx + row * a.s.max_kb;
+  }
+  return ok;
+}
+
 // OUTP: the output goes through the K/V page table (FP_OUT_PAGED; paged K/V only). A template
 // parameter, so that the other instantiations keep no page-table state live through the loop.
-template <int D, int BN, bool FP8, bool PAGED, bool OUTP>
+// QP: the general work split (query-block pairs, tiles of two requests); without it the
+// head-pair split, whose tiles share one request.
+template <int D, int BN, bool FP8, bool PAGED, bool OUTP, bool QP>
 __global__ void __launch_bounds__(384, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
@@ -166,9 +245,12 @@ __global__ void __launch_bounds__(384, 1)
   if (sh.abort_flag) return;
 
   Tile tl[2];
-  int g, b, kbase, len;
-  if (!make_tiles(a, blockIdx.x, tl, g, b, kbase, len) && threadIdx.x == 0)
-    record_status(a.status, kStatusBadIndex);
+  Req rq[2];
+  int g, b = 0, kbase = 0, len = 0;
+  bool tiles_ok;
+  if constexpr (QP) tiles_ok = make_tiles_qp(a, blockIdx.x, tl, rq, g);
+  else tiles_ok = make_tiles(a, blockIdx.x, tl, g, b, kbase, len);
+  if (!tiles_ok && threadIdx.x == 0) record_status(a.status, kStatusBadIndex);
   // Producer bookkeeping: the last use of each ring slot whose load was issued, so that a CTA
   // that gives up waits (bounded) for its own bulk copies before it exits.
   int k_issued[C::kKSt], v_issued[C::kVSt];
@@ -214,8 +296,8 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_3d(smem + C::kQOff + s * C::kQBytes + c * (C::kBM * 128), &tm_q, &sh.q_full,
                       c * C::kChunkEl, tl[s].h, tl[s].q_lo);
       q_issued = true;
-      UnionWalk uw;
-      uw.init(tl[0], tl[1]);
+      UnionWalk<QP> uw;
+      uw.init(tl[0], tl[1], rq[0].kb0, rq[1].kb0);
       int J, bits;
       for (int k = 0; uw.next(J, bits); ++k) {
         if (sh.abort_flag) break;
@@ -224,6 +306,15 @@ __global__ void __launch_bounds__(384, 1)
         constexpr int kSegRows = PAGED ? 0 : BN;
         const int seg_rows = PAGED ? a.page_size : kSegRows;
         const int nseg = BN / seg_rows;
+        // The block's request (with QP the tiles' requests may differ, and then no block has
+        // bits = 3).
+        int kb_req = kbase, len_req = len, b_req = b;
+        if constexpr (QP) {
+          const bool from0 = bits & 1;
+          kb_req = from0 ? rq[0].kbase : rq[1].kbase;
+          len_req = from0 ? rq[0].len : rq[1].len;
+          b_req = from0 ? rq[0].b : rq[1].b;
+        }
         for (int which = 0; which < 2; ++which) {
           const int st = which == 0 ? ks : vs;
           uint64_t* full = which == 0 ? &sh.k_full[st] : &sh.v_full[st];
@@ -242,16 +333,16 @@ __global__ void __launch_bounds__(384, 1)
             int row;
             const int tok = J * BN + sgi * seg_rows;  // request-local first token
             if constexpr (PAGED) {
-              const int pages_req = (len + a.page_size - 1) / a.page_size;
+              const int pages_req = (len_req + a.page_size - 1) / a.page_size;
               const int lp = tok / a.page_size;
               row = a.num_pages * a.page_size;  // past the end: TMA fills zeros
               if (lp < pages_req && lp < a.max_pages) {
-                const int pid = __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp);
+                const int pid = __ldg(a.page_table + static_cast<size_t>(b_req) * a.max_pages + lp);
                 if (pid >= 0 && pid < a.num_pages) row = pid * a.page_size;
                 else record_status(a.status, kStatusBadIndex);
               }
             } else {
-              row = kbase + tok;
+              row = kb_req + tok;
             }
             for (int c = 0; c < C::kNChunk; ++c)
               tma_load_3d(dst + c * (BN * 128) + sgi * (seg_rows * 128), tm, full,
@@ -295,8 +386,8 @@ __global__ void __launch_bounds__(384, 1)
         pend[t] = -1;
         return true;
       };
-      UnionWalk uw;
-      uw.init(tl[0], tl[1]);
+      UnionWalk<QP> uw;
+      uw.init(tl[0], tl[1], rq[0].kb0, rq[1].kb0);
       int J, bits;
       for (int k = 0; ok && uw.next(J, bits); ++k) {
         if (sh.abort_flag) { ok = false; break; }
@@ -479,10 +570,12 @@ __global__ void __launch_bounds__(384, 1)
       bool valid = r >= T.r0 && r < T.r1;
       size_t out_row = static_cast<size_t>(T.q_lo + r);
       if (OUTP && valid) {
+        int b_out = b;
+        if constexpr (QP) b_out = t == 0 ? rq[0].b : rq[1].b;
         const int pos = T.I * BN + r;
         const int lp = pos / a.page_size;
         const int pg = lp < a.max_pages
-                           ? __ldg(a.page_table + static_cast<size_t>(b) * a.max_pages + lp) : -1;
+                           ? __ldg(a.page_table + static_cast<size_t>(b_out) * a.max_pages + lp) : -1;
         if (pg >= 0 && pg < a.num_pages) {
           out_row = static_cast<size_t>(pg) * a.page_size + pos % a.page_size;
         } else {
@@ -564,21 +657,29 @@ static bool make_map(CUtensorMap* m, const void* base, bool e4m3, int d, int hea
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool OUTP = false>
-static cudaError_t launch_t(const AttnArgs& a, const AttnLaunch& L, cudaStream_t stream) {
+template <int D, int BN, bool FP8, bool PAGED, bool OUTP, bool QP>
+static cudaError_t launch_s(const AttnArgs& a, const AttnLaunch& L, cudaStream_t stream) {
   using C = AttnCfg<D, BN, FP8>;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, L.q, FP8, D, a.Hq, a.s.total_q, 128) ||
       !make_map(&mk, L.k, FP8, D, a.Hkv, L.kv_rows, L.seg_rows) ||
       !make_map(&mv, L.v, FP8, D, a.Hkv, L.kv_rows, L.seg_rows))
     return cudaErrorInvalidValue;
-  auto kern = attn_kernel<D, BN, FP8, PAGED, OUTP>;
+  auto kern = attn_kernel<D, BN, FP8, PAGED, OUTP, QP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (a.num_items == 0) return cudaSuccess;
   kern<<<a.num_items, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, a);
   return cudaGetLastError();
+}
+
+// Work split: the head-pair kernel unless some head pairs query blocks (G odd, G = 1,
+// FP_PAIR_QBLOCKS).
+template <int D, int BN, bool FP8, bool PAGED, bool OUTP = false>
+static cudaError_t launch_t(const AttnArgs& a, const AttnLaunch& L, cudaStream_t stream) {
+  return a.qpair_heads > 0 ? launch_s<D, BN, FP8, PAGED, OUTP, true>(a, L, stream)
+                           : launch_s<D, BN, FP8, PAGED, OUTP, false>(a, L, stream);
 }
 
 // Paged K/V: with the paged output layout or without it.

@@ -68,7 +68,9 @@ struct AttnArgs {
   int Hq, Hkv;
   int page_size, max_pages, num_pages;  // paged only
   int G;                               // query heads per KV head
-  int num_items;                        // Hkv * ceil(G / 2) * total_qb
+  int head_pairs;                       // per KV head: head pairs (two heads, one query block)
+  int qpair_heads;                      // per KV head: heads paired over two query blocks
+  int num_items;                        // CTAs: levels of two query blocks (see attn.cu)
   int fault_skip_k;                     // test hook: CTA 0 skips the K load of this union block
   int out_paged;                        // out is [num_pages, page_size, Hq, d] via page_table
   float scale_log2;                     // softmax scale * log2(e)

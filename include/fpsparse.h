@@ -77,10 +77,14 @@ extern "C" {
 
 #define FP_OUT_PAGED 1   /* out_flags of fp_sparse_prefill_attn_chunked: write O in the paged
                             layout of the K/V cache (see there) */
+#define FP_PAIR_QBLOCKS 2 /* out_flags of fp_sparse_prefill_attn_chunked: every CTA pairs two
+                            neighbouring query blocks of one head instead of two heads of a GQA
+                            group (see the work split under fp_sparse_prefill_attn) */
 
-/* Library version, e.g. 200 for 0.2.0. 0.1.1 added the chunked-prefill calls, the paged K/V
+/* Library version, e.g. 300 for 0.3.0. 0.1.1 added the chunked-prefill calls, the paged K/V
  * append and FP_MASK_FP32; 0.2.0 gives the pool and mask calls a workspace (status word) and
- * checks the prefix sums on the device. */
+ * checks the prefix sums on the device; 0.3.0 pairs query blocks where heads cannot be paired
+ * (G = 1, the last head of an odd G) and adds FP_PAIR_QBLOCKS. */
 int fp_version(void);
 
 /* Message describing the last error returned on the calling thread ("" if none). */
@@ -170,6 +174,13 @@ int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_
  *            workspaces.
  * Supported: d in {64, 128}; block in {64, 128} (e4m3: d = 128, block = 128);
  * Hq % Hkv == 0. Q, K, V must be 16-byte aligned.
+ * Work split (the output is bit-identical whichever split runs: every tile accumulates its own
+ * kept blocks in ascending order with the same instructions): each CTA runs two query tiles
+ * that read the same KV head and loads every KV block either tile kept once. With G = Hq / Hkv
+ * even, the tiles are two heads of a GQA group at one query block; the head an odd G leaves
+ * over, and every head when G = 1, is paired with itself over two neighbouring query blocks
+ * (cross-query reuse, "QUILT: Rethinking Sparse-Attention Prefill through Shared Query
+ * Execution", Abstract). FP_PAIR_QBLOCKS (chunked call) pairs query blocks for every head.
  */
 int fp_sparse_prefill_attn(const void* q, const void* k, const void* v, int dtype,
                            const float* q_scale, const float* k_scale, const float* v_scale,
@@ -239,8 +250,9 @@ int fp_sparse_prefill_attn_paged(const void* q, const void* k_cache, const void*
  * needed to place query blocks (64 or 128).
  * fp_sparse_prefill_attn_chunked: out [total_q, Hq, d] bf16 and lse [Hq, total_q] (or NULL) for
  * the queries only. K and V are contiguous [total_k, Hkv, d] (page_table NULL) or caches read
- * through page_table (same rules as fp_sparse_prefill_attn_paged). out_flags is 0 or
- * FP_OUT_PAGED: then out is instead a bf16 buffer [num_pages, page_size, Hq, d] in the page
+ * through page_table (same rules as fp_sparse_prefill_attn_paged). out_flags is a
+ * combination of FP_PAIR_QBLOCKS (the work split above; the output is the same) and
+ * FP_OUT_PAGED: with FP_OUT_PAGED out is instead a bf16 buffer [num_pages, page_size, Hq, d] in the page
  * layout of the K/V caches, and the output row of the query at absolute position p of request
  * b goes to slot p % page_size of page page_table[b * max_pages + p / page_size] (the page
  * table must be given; an entry out of range skips the row and records FP_ERR_BAD_INDEX; slots

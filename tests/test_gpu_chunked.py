@@ -36,6 +36,9 @@ CASES = {
     "b64_d64": (dataclasses.replace(BASE, block=64, d=64), (700, 333), (250, 90), 0.5),
     "gqa3": (dataclasses.replace(BASE, Hq=6), (800, 500), (300, 77), 0.5),
     "gqa5": (dataclasses.replace(BASE, Hq=10, structure="band"), (900, 1300), (450, 129), 0.1),
+    # one query head per KV head: query-block pairs. 6 + 7 + 2 query blocks: the pair (6, 5)
+    # holds the first block of request 1 and the last of request 0
+    "mha": (dataclasses.replace(BASE, Hq=2, Hkv=2), (1000, 850, 300), (744, 850, 65), 0.5),
     # many key blocks per row (several score chunks in the mask kernel), long cached prefix
     "long_prefix": (dataclasses.replace(W["llama128k"], Hq=8, Hkv=2), (20000, 9000),
                     (1500, 2700), 0.1),
@@ -276,3 +279,37 @@ def test_paged_output_layout_equals_the_contiguous_output(name, cuda_device):
         written.view(-1)[slots] = True
     rest = pages.view(-1, w.Hq, w.d)[~written.view(-1).to(cuda_device)]
     assert bool((rest == 5.0).all())
+
+
+@pytest.mark.parametrize("name", ["mixed", "paged", "fp8", "b64_d64", "gqa3", "gqa5", "mha",
+                                  "long_prefix", "paged_out"])
+def test_query_block_pairing_gives_the_same_output(name, cuda_device):
+    """FP_PAIR_QBLOCKS: every CTA runs one head over two neighbouring query blocks (both tiles
+    read each KV block they both kept once) instead of two heads of a GQA group at one query
+    block. Each tile still accumulates its own kept blocks in ascending order with the same
+    instructions, so out and lse equal the default split's bit for bit, for pairs inside a
+    request and across request boundaries, contiguous or paged K/V, bf16 or e4m3."""
+    inp, alpha = _inputs("paged" if name == "paged_out" else name)
+    q, k, v, sc = device_inputs(inp, cuda_device)
+    cb = _cb(inp, cuda_device)
+    paged = _paged(inp, cuda_device)
+    kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"],
+              return_lse=True, paged=paged)
+    kk, vv = (None, None) if paged is not None else (k, v)
+    qp, kp = fp.pool_qk_chunked(q, kk, cb, q_scale=sc["q_scale"], k_scale=sc["k_scale"],
+                                paged=paged)
+    _, cnt, idx = fp.build_block_mask_chunked(qp, kp, cb, alpha, mask_bits=False)
+    out_paged = name == "paged_out"
+    outs = []
+    for pair in (False, True):
+        out = None
+        if out_paged:
+            out = torch.full((paged.k_cache.shape[0], paged.page_size, q.shape[1], q.shape[2]),
+                             5.0, dtype=torch.bfloat16, device=cuda_device)
+        outs.append(fp.sparse_prefill_attn_chunked(q, kk, vv, cnt, idx, cb, out=out,
+                                                   out_paged=out_paged, pair_qblocks=pair,
+                                                   **kw))
+    fp.check_status(cuda_device)
+    (o0, l0), (o1, l1) = outs
+    assert torch.equal(o0, o1)
+    assert torch.equal(l0, l1)

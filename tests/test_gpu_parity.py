@@ -64,6 +64,18 @@ def _case(name):
                          (300, 0, 129), 0.5),
         "paged_empty": (dataclasses.replace(W["paged"], Hq=8, Hkv=2, structure="iid"),
                         (0, 200, 0, 65), 0.5),
+        # one query head per KV head: every CTA pairs two neighbouring query blocks of a head.
+        # 3 + 2 + 5 query blocks: pairs (5, 4) and (3, 2) straddle request boundaries (the two
+        # tiles read different requests' K/V); 3 + 2 + 5 + 1 blocks leave a last single tile
+        "mha_varlen": (dataclasses.replace(base, Hq=2, Hkv=2, structure="iid"),
+                       (300, 129, 640), 0.5),
+        "mha_paged": (dataclasses.replace(W["paged"], Hq=2, Hkv=2, structure="iid"),
+                      (300, 129, 640, 77), 0.5),
+        "mha_fp8": (dataclasses.replace(W["fp8_128k"], Hq=3, Hkv=3, structure="iid"),
+                    (300, 129, 640, 77), 0.5),
+        # odd G with varlen: the third head of each group pairs query blocks across requests
+        "gqa3_varlen": (dataclasses.replace(base, Hq=6, Hkv=2, structure="band"),
+                        (300, 129, 640, 77), 0.1),
     }
     w, seqlens, alpha = cases[name]
     return S.make_inputs(w, seed=7, seqlens=seqlens), alpha
@@ -71,7 +83,8 @@ def _case(name):
 
 SMALL = ["tiny", "tiny_a09", "gqa_ragged", "gqa_ragged_a05", "varlen", "paged", "fp8",
          "mha_d128", "dense_alpha0", "d128_b64", "d64_b128", "long_ragged", "varlen_long", "gqa8",
-         "gqa3", "gqa5", "gqa7", "gqa5_iid", "gqa7_iid", "varlen_empty", "paged_empty"]
+         "gqa3", "gqa5", "gqa7", "gqa5_iid", "gqa7_iid", "varlen_empty", "paged_empty", "mha_varlen",
+         "mha_paged", "mha_fp8", "gqa3_varlen"]
 # cases whose full fp64 attention would be slow: the oracle runs on every 5th query block
 SAMPLED = {"long_ragged", "varlen_long"}
 
