@@ -303,16 +303,18 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
   a.num_pages = num_pages;
   a.G = G;
   // Two heads of a GQA group per CTA; a head left over (odd G, all heads for G = 1, or every
-  // head with FP_PAIR_QBLOCKS) pairs two neighbouring query blocks instead. Per level of two
-  // query blocks: Hkv * head_pairs items at each block and Hkv * qpair_heads items over both;
-  // for an odd total_qb the last level has no second block and its head pairs are not launched.
+  // head with FP_PAIR_QBLOCKS) pairs two neighbouring query blocks instead. Head pairs alone:
+  // Hkv * G / 2 items per query block. Otherwise per level of two query blocks and KV head,
+  // head_pairs items at each block and qpair_heads over both (at the last level of an odd
+  // total_qb the second block's head pairs have no work and end at once).
   a.head_pairs = (out_flags & FP_PAIR_QBLOCKS) ? 0 : G / 2;
   a.qpair_heads = G - 2 * a.head_pairs;
   {
     const long long levels = (static_cast<long long>(s.total_qb) + 1) / 2;
-    const long long per_level = static_cast<long long>(Hkv) * (2 * a.head_pairs + a.qpair_heads);
     const long long items =
-        levels * per_level - ((s.total_qb & 1) ? static_cast<long long>(Hkv) * a.head_pairs : 0);
+        a.qpair_heads == 0
+            ? static_cast<long long>(Hkv) * a.head_pairs * s.total_qb
+            : levels * Hkv * (2 * a.head_pairs + a.qpair_heads);
     if (items > INT_MAX) return fail(FP_ERR_INVALID_ARG, "too many attention work items");
     a.num_items = static_cast<int>(items);
   }

@@ -73,6 +73,9 @@ struct Req {
   int b, kbase, len, kb0;
 };
 
+// Levels (pairs of query blocks) per item window of the general work split (make_tiles_qp).
+constexpr int kQpWindow = 32;
+
 struct Shared {  // placed at kBarOff
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];  // ring slots (kKSt, kVSt <= 4)
@@ -160,34 +163,38 @@ __device__ __forceinline__ bool make_tiles(const AttnArgs& a, int item, Tile* t,
   return qb.ok;
 }
 
-// General split: work item -> two tiles that read the same KV head. Two heads of a GQA group share a query
-// block (a head pair); a head that pairing leaves over (odd G, every head when G = 1, or every
-// head when query-block pairing is forced) is paired with itself over two neighbouring query
-// blocks (the QUILT page's cross-query reuse: both tiles read every block they both kept once).
-// Items run heaviest-first in levels of two query blocks, Ig0 = total_qb - 1 - 2 * level and
-// Ig1 = Ig0 - 1: per level Hkv * hp head pairs at Ig0, Hkv * nqh query-block pairs, then
-// Hkv * hp head pairs at Ig1 (absent at the last level when total_qb is odd, so the host
-// launches none of them). Returns false (tiles absent) when the prefix sums do not describe a
-// tile's request consistently.
+// General split: work item -> two tiles that read the same KV head. Two heads of a GQA group
+// share a query block (a head pair); a head that pairing leaves over (odd G, every head when
+// G = 1, or every head when query-block pairing is forced) is paired with itself over two
+// neighbouring query blocks (the QUILT page's cross-query reuse: both tiles read every block
+// they both kept once). Levels of two query blocks, Ig0 = total_qb - 1 - 2 * level and
+// Ig1 = Ig0 - 1, hold per KV head S = 2 hp + nqh items: hp head pairs at Ig0, nqh query-block
+// pairs, hp head pairs at Ig1 (both tiles absent at the last level when total_qb is odd).
+// Items run heaviest-first in windows of kQpWindow levels, and inside a window KV head by KV
+// head: the CTAs in flight (about one per SM) then cover a few KV heads over many neighbouring
+// query blocks, so the K/V blocks those share (the local band, columns every row keeps) stay in
+// L2 instead of every KV head's working set at once. Returns false (tiles absent) when the
+// prefix sums do not describe a tile's request consistently.
 __device__ __forceinline__ bool make_tiles_qp(const AttnArgs& a, int item, Tile* t, Req* rq,
                                               int& g) {
-  const int hp = a.head_pairs, nqh = a.qpair_heads;
-  const int nA = a.Hkv * hp, nB = a.Hkv * nqh;
-  const int level = item / (2 * nA + nB);
-  int rem = item % (2 * nA + nB);
-  const int Ig0 = a.s.total_qb - 1 - 2 * level;
+  const int hp = a.head_pairs, nqh = a.qpair_heads, S = 2 * hp + nqh;
+  const int levels = (a.s.total_qb + 1) / 2;
+  const int per_win = kQpWindow * a.Hkv * S;
+  const int win = item / per_win;
+  int rem = item % per_win;
+  const int wn = min(kQpWindow, levels - win * kQpWindow);  // levels in this window
+  g = rem / (wn * S);
+  rem %= wn * S;
+  const int Ig0 = a.s.total_qb - 1 - 2 * (win * kQpWindow + rem / S);
+  const int slot = rem % S;
   int Igs[2];
-  if (rem < nA || rem >= nA + nB) {
-    const bool second = rem >= nA;
-    if (second) rem -= nA + nB;
-    g = rem / hp;
-    t[0].h = g * a.G + 2 * (rem % hp);
+  if (slot < hp || slot >= hp + nqh) {
+    const bool second = slot >= hp;
+    t[0].h = g * a.G + 2 * (second ? slot - hp - nqh : slot);
     t[1].h = t[0].h + 1;
     Igs[0] = Igs[1] = second ? Ig0 - 1 : Ig0;
   } else {
-    rem -= nA;
-    g = rem / nqh;
-    t[0].h = t[1].h = g * a.G + 2 * hp + rem % nqh;
+    t[0].h = t[1].h = g * a.G + 2 * hp + (slot - hp);
     Igs[0] = Ig0;
     Igs[1] = Ig0 - 1;
   }
@@ -251,6 +258,10 @@ __global__ void __launch_bounds__(384, 1)
   if constexpr (QP) tiles_ok = make_tiles_qp(a, blockIdx.x, tl, rq, g);
   else tiles_ok = make_tiles(a, blockIdx.x, tl, g, b, kbase, len);
   if (!tiles_ok && threadIdx.x == 0) record_status(a.status, kStatusBadIndex);
+  // A head pair past the first query block (odd total_qb, last level) has no work; every
+  // thread of the CTA maps the same item, so the whole CTA leaves together.
+  if constexpr (QP)
+    if (tl[0].Ig < 0 && tl[1].Ig < 0) return;
   // Producer bookkeeping: the last use of each ring slot whose load was issued, so that a CTA
   // that gives up waits (bounded) for its own bulk copies before it exits.
   int k_issued[C::kKSt], v_issued[C::kVSt];
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(384, 1)
                       c * C::kChunkEl, tl[s].h, tl[s].q_lo);
       q_issued = true;
       UnionWalk<QP> uw;
-      uw.init(tl[0], tl[1], rq[0].kb0, rq[1].kb0);
+      uw.init(tl[0], tl[1], QP ? rq[0].kb0 : 0, QP ? rq[1].kb0 : 0);
       int J, bits;
       for (int k = 0; uw.next(J, bits); ++k) {
         if (sh.abort_flag) break;
@@ -387,7 +398,7 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       UnionWalk<QP> uw;
-      uw.init(tl[0], tl[1], rq[0].kb0, rq[1].kb0);
+      uw.init(tl[0], tl[1], QP ? rq[0].kb0 : 0, QP ? rq[1].kb0 : 0);
       int J, bits;
       for (int k = 0; ok && uw.next(J, bits); ++k) {
         if (sh.abort_flag) { ok = false; break; }

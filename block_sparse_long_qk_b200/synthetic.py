@@ -1,6 +1,6 @@
 """Seeded synthetic workloads for block-sparse causal prefill attention.
 
-This module draws the random inputs that the six workloads are described with and casts
+This module draws the random inputs that the seven workloads are described with and casts
 them to the storage types the kernels read (bf16, or e4m3 with per-head absmax scales).
 It holds none of the method's own arithmetic (no pooling, scoring, thresholding or
 attention), so it can feed both the CUDA path and the fp64 oracle without coupling them.
@@ -19,6 +19,8 @@ summary section 4):
                added, times BAND_AMPLITUDE, to K[t, g] and to Q[t, h] of the query heads
                h that read g. V ~ N(0,1).
 * ``fp8_128k`` the ``llama128k`` tensors quantised per head to e4m3 (scale = absmax/448).
+* ``mha128k``  the ``llama128k`` recipe with one query head per KV head (Hq = Hkv = 32:
+               multi-head attention, where no two query heads share K/V).
 * ``paged``    8 requests, lengths uniform in [4096, 65536], each drawn with the
                ``llama128k`` recipe under its own seed; K/V stored in 64-token pages
                whose physical order is a seeded random permutation.
@@ -96,6 +98,7 @@ WORKLOADS = {
     "llama128k": Workload("llama128k", (131072,), 32, 8, 128, 128, structure="band"),
     "fp8_128k": Workload("fp8_128k", (131072,), 32, 8, 128, 128, dtype="e4m3",
                          structure="band"),
+    "mha128k": Workload("mha128k", (131072,), 32, 32, 128, 128, structure="band"),
     "paged": Workload("paged", paged_lengths(1234 + 5), 32, 8, 128, 128, structure="band",
                       page_size=64),
     "chunked": Workload("chunked", _CHUNKED_KV, 32, 8, 128, 128, structure="band",
@@ -103,7 +106,7 @@ WORKLOADS = {
 }
 
 DEFAULT_SEEDS = {"tiny": 1235, "llama32k": 1236, "llama128k": 1237, "fp8_128k": 1237,
-                 "paged": 1239, "chunked": 1240}
+                 "paged": 1239, "chunked": 1240, "mha128k": 1241}
 
 
 def _normal(seed_seq: np.random.SeedSequence, shape) -> np.ndarray:

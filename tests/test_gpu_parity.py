@@ -320,7 +320,8 @@ def _full_size(name, cuda_device):
     return run
 
 
-@pytest.mark.parametrize("name", ["llama32k", "llama128k", "fp8_128k", "paged", "chunked"])
+@pytest.mark.parametrize("name", ["llama32k", "llama128k", "fp8_128k", "paged", "chunked",
+                                  "mha128k"])
 def test_full_size_workloads(name, cuda_device):
     _full_size(name, cuda_device)
 
