@@ -308,7 +308,8 @@ __global__ void __launch_bounds__(384, 1)
                       c * C::kChunkEl, tl[s].h, tl[s].q_lo);
       q_issued = true;
       UnionWalk<QP> uw;
-      uw.init(tl[0], tl[1], QP ? rq[0].kb0 : 0, QP ? rq[1].kb0 : 0);
+      if constexpr (QP) uw.init(tl[0], tl[1], rq[0].kb0, rq[1].kb0);
+      else uw.init(tl[0], tl[1]);
       int J, bits;
       for (int k = 0; uw.next(J, bits); ++k) {
         if (sh.abort_flag) break;
@@ -398,7 +399,8 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       UnionWalk<QP> uw;
-      uw.init(tl[0], tl[1], QP ? rq[0].kb0 : 0, QP ? rq[1].kb0 : 0);
+      if constexpr (QP) uw.init(tl[0], tl[1], rq[0].kb0, rq[1].kb0);
+      else uw.init(tl[0], tl[1]);
       int J, bits;
       for (int k = 0; ok && uw.next(J, bits); ++k) {
         if (sh.abort_flag) { ok = false; break; }
