@@ -1,5 +1,6 @@
 // extern "C" entry points of libfpsparse.so: argument checks, then one kernel launch each.
 // Declarations and the contract of every call are in include/fpsparse.h.
+#include <atomic>
 #include <limits.h>
 #include <math.h>
 #include <stdarg.h>
@@ -264,6 +265,20 @@ int mask_impl(const float* q_pool, const float* k_pool, const void* k_pool_split
   return e == cudaSuccess ? FP_OK : cuda_fail(e, "mask kernel launch");
 }
 
+// SMs of the calling thread's current device (cached per device; 148 if the query fails).
+int device_sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
 int attn_impl(const void* q, const void* k, const void* v, int dtype, const float* q_scale,
               const float* k_scale, const float* v_scale, const fp::Seqs& s, int Hq, int Hkv,
               int d, const int32_t* page_table, int page_size, int max_pages, int num_pages,
@@ -302,19 +317,24 @@ int attn_impl(const void* q, const void* k, const void* v, int dtype, const floa
   a.max_pages = max_pages;
   a.num_pages = num_pages;
   a.G = G;
-  // Two heads of a GQA group per CTA; a head left over (odd G, all heads for G = 1, or every
-  // head with FP_PAIR_QBLOCKS) pairs two neighbouring query blocks instead. Head pairs alone:
-  // Hkv * G / 2 items per query block. Otherwise per level of two query blocks and KV head,
-  // head_pairs items at each block and qpair_heads over both (at the last level of an odd
-  // total_qb the second block's head pairs have no work and end at once).
+  // Two heads of a GQA group per CTA. A head left over (odd G, all heads for G = 1) runs alone
+  // in its CTA or pairs two neighbouring query blocks: pairing halves those heads' CTAs and
+  // makes each ~1.2x longer, which pays once their single tiles would fill the GPU at least
+  // twice (with fewer, SMs would idle); FP_PAIR_QBLOCKS pairs query blocks for every head.
+  // Head-pair kernel: Hkv * ceil(G / 2) items per query block (the odd head alone). General
+  // split: per level of two query blocks and KV head, head_pairs items at each block and
+  // qpair_heads over both (at the last level of an odd total_qb the second block's head pairs
+  // have no work and end at once).
+  const long long single_items = static_cast<long long>(Hkv) * ((G + 1) / 2) * s.total_qb;
+  const bool pair_q = (out_flags & FP_PAIR_QBLOCKS) ||
+                      (G % 2 == 1 && single_items >= 2LL * device_sm_count());
   a.head_pairs = (out_flags & FP_PAIR_QBLOCKS) ? 0 : G / 2;
-  a.qpair_heads = G - 2 * a.head_pairs;
+  a.qpair_heads = pair_q ? G - 2 * a.head_pairs : 0;
   {
     const long long levels = (static_cast<long long>(s.total_qb) + 1) / 2;
     const long long items =
-        a.qpair_heads == 0
-            ? static_cast<long long>(Hkv) * a.head_pairs * s.total_qb
-            : levels * Hkv * (2 * a.head_pairs + a.qpair_heads);
+        a.qpair_heads == 0 ? single_items
+                           : levels * Hkv * (2 * a.head_pairs + a.qpair_heads);
     if (items > INT_MAX) return fail(FP_ERR_INVALID_ARG, "too many attention work items");
     a.num_items = static_cast<int>(items);
   }

@@ -123,15 +123,15 @@ struct UnionWalk {
   }
 };
 
-// Head-pair split (G even): work item -> two heads of a GQA group at one query block, one
-// request. Items run heaviest-first (late query blocks have the longest causal rows). `kbase`
+// Head-pair split: work item -> two heads of a GQA group at one query block, one request. Items run heaviest-first (late query blocks have the longest causal rows). `kbase`
 // / `len`: key row of the request's position 0 and its key count; `b`: the request (page-table
 // row). Returns false (both tiles absent) when the prefix sums do not describe the request
 // consistently.
 __device__ __forceinline__ bool make_tiles(const AttnArgs& a, int item, Tile* t, int& g,
                                            int& b, int& kbase, int& len) {
-  // The G query heads of a KV head form G / 2 items per query block, pairs of heads (the
-  // general split below takes odd G; for it, this mapping would leave the last head alone).
+  // The G query heads of a KV head form ceil(G / 2) items per query block: pairs of heads,
+  // and for an odd G one single head (its CTA runs one tile; the host sends an odd G here only
+  // when single tiles give the GPU more CTAs than it could otherwise fill).
   const int npair = (a.G + 1) / 2;
   const int per_block = a.Hkv * npair;
   const int Ig = a.s.total_qb - 1 - item / per_block;
@@ -687,8 +687,8 @@ static cudaError_t launch_s(const AttnArgs& a, const AttnLaunch& L, cudaStream_t
   return cudaGetLastError();
 }
 
-// Work split: the head-pair kernel unless some head pairs query blocks (G odd, G = 1,
-// FP_PAIR_QBLOCKS).
+// Work split: the head-pair kernel unless some head pairs query blocks (odd G or G = 1 on
+// problems large enough, or FP_PAIR_QBLOCKS).
 template <int D, int BN, bool FP8, bool PAGED, bool OUTP = false>
 static cudaError_t launch_t(const AttnArgs& a, const AttnLaunch& L, cudaStream_t stream) {
   return a.qpair_heads > 0 ? launch_s<D, BN, FP8, PAGED, OUTP, true>(a, L, stream)

@@ -180,7 +180,9 @@ int fp_build_block_mask(const float* q_pool, const float* k_pool, const void* k_
  * even, the tiles are two heads of a GQA group at one query block; the head an odd G leaves
  * over, and every head when G = 1, is paired with itself over two neighbouring query blocks
  * (cross-query reuse, "QUILT: Rethinking Sparse-Attention Prefill through Shared Query
- * Execution", Abstract). FP_PAIR_QBLOCKS (chunked call) pairs query blocks for every head.
+ * Execution", Abstract) when those heads' single tiles would fill the GPU's SMs at least twice,
+ * and runs one tile per CTA on smaller problems. FP_PAIR_QBLOCKS (chunked call) pairs query
+ * blocks for every head.
  */
 int fp_sparse_prefill_attn(const void* q, const void* k, const void* v, int dtype,
                            const float* q_scale, const float* k_scale, const float* v_scale,

@@ -64,16 +64,16 @@ def _case(name):
                          (300, 0, 129), 0.5),
         "paged_empty": (dataclasses.replace(W["paged"], Hq=8, Hkv=2, structure="iid"),
                         (0, 200, 0, 65), 0.5),
-        # one query head per KV head: every CTA pairs two neighbouring query blocks of a head.
-        # 3 + 2 + 5 query blocks: pairs (5, 4) and (3, 2) straddle request boundaries (the two
-        # tiles read different requests' K/V); 3 + 2 + 5 + 1 blocks leave a last single tile
+        # one query head per KV head (and below, an odd group): at these sizes each CTA runs a
+        # single tile (query-block pairs, which straddle request boundaries in these length
+        # mixes, are taken on problems of two waves or more: `mha128k` at full size, and the
+        # FP_PAIR_QBLOCKS tests of test_gpu_chunked.py on small ones)
         "mha_varlen": (dataclasses.replace(base, Hq=2, Hkv=2, structure="iid"),
                        (300, 129, 640), 0.5),
         "mha_paged": (dataclasses.replace(W["paged"], Hq=2, Hkv=2, structure="iid"),
                       (300, 129, 640, 77), 0.5),
         "mha_fp8": (dataclasses.replace(W["fp8_128k"], Hq=3, Hkv=3, structure="iid"),
                     (300, 129, 640, 77), 0.5),
-        # odd G with varlen: the third head of each group pairs query blocks across requests
         "gqa3_varlen": (dataclasses.replace(base, Hq=6, Hkv=2, structure="band"),
                         (300, 129, 640, 77), 0.1),
     }
