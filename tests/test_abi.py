@@ -162,11 +162,24 @@ def _bad_chunked_attn(**over):
     (dict(pt=16, ps=48), -1),        # page size not dividing the block
     (dict(dtype=1, qs=16, ks=16, vs=16, d=64), -2),   # e4m3 needs d = 128
     (dict(of=1), -1),                # paged output without a page table
-    (dict(of=2), -1),                # unknown output flag
+    (dict(of=3), -1),                # the same with query-block pairing (FP_PAIR_QBLOCKS = 2)
+    (dict(of=4), -1),                # unknown flag
 ])
 def test_chunked_attention_rejects_bad_arguments(over, code):
     assert _bad_chunked_attn(**over) == code
     assert fp.library().fp_last_error_string()
+
+
+def test_chunked_attention_flag_messages():
+    """FP_OUT_PAGED (1) and FP_PAIR_QBLOCKS (2) are the only flags; any other bit is refused
+    as unknown, and the paged output is refused for its missing page table, not its flag."""
+    assert fp.OUT_PAGED == 1 and fp.PAIR_QBLOCKS == 2
+    for of in (4, 8, 1 << 30):
+        assert _bad_chunked_attn(of=of) == -1
+        assert b"unknown flags" in fp.library().fp_last_error_string()
+    for of in (1, 3):
+        assert _bad_chunked_attn(of=of) == -1
+        assert b"page table" in fp.library().fp_last_error_string()
 
 
 def test_chunked_mask_and_pool_reject_bad_arguments():
