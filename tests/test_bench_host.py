@@ -59,3 +59,18 @@ def test_head_pairs_share_more_kept_blocks_than_query_block_pairs():
     assert nq % 2 == 0
     assert qblk_union > 1.02 * head_union
     assert head_union < 0.51 * int(K.sum())      # the two heads' lists nearly coincide
+
+
+def test_every_full_size_workload_has_a_traffic_figure():
+    """bench.py reports the attention kernel's measured DRAM bytes per launch as
+    roofline.traffic; every workload bench.py can run at full size has its figure (the tiny
+    layer fits in L2 and reports none)."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                           "profiles", "attn_traffic.json")) as f:
+        traffic = json.load(f)
+    for name in S.WORKLOADS:
+        if name == "tiny":
+            continue
+        assert name in traffic and traffic[name] > 0, name
