@@ -69,8 +69,9 @@ struct AttnArgs {
   int page_size, max_pages, num_pages;  // paged only
   int G;                               // query heads per KV head
   int head_pairs;                       // per KV head: head pairs (two heads, one query block)
-  int qpair_heads;                      // per KV head: heads paired over two query blocks
-  int num_items;                        // CTAs: levels of two query blocks (see attn.cu)
+  int qpair_heads;                      // per KV head: heads paired over two query blocks; 0
+                                        // selects the head-pair kernel (odd G: last head alone)
+  int num_items;                        // CTAs (make_tiles / make_tiles_qp in attn.cu)
   int fault_skip_k;                     // test hook: CTA 0 skips the K load of this union block
   int out_paged;                        // out is [num_pages, page_size, Hq, d] via page_table
   float scale_log2;                     // softmax scale * log2(e)
