@@ -374,10 +374,12 @@ def time_layer(layer, steps, warmup, world, dev, local):
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    # A ~25 ms device-side spin ahead of the start event lets the host enqueue the timed steps
-    # before the GPU reaches them, so a host-side stall while launching cannot leave the GPU
-    # idle inside the timed region (the events would count that idle time).
-    torch.cuda._sleep(50_000_000)
+    # A device-side spin ahead of the start event (25 ms plus 1 ms per timed step, at 2 GHz;
+    # longer at the lower clocks the power cap sets) lets the host enqueue every timed step
+    # before the GPU reaches them, so a host-side stall while launching (a launch that waits
+    # for the driver, e.g. while the clock sampler queries it) cannot leave the GPU idle inside
+    # the timed region: the events would count that idle time.
+    torch.cuda._sleep(2_000_000 * (25 + steps))
     t_start.record()
     for i in range(steps):
         out, cnt, idx = layer.step(evs[i])
@@ -434,8 +436,9 @@ def roofline(w, alg, executed, attn_ms, peaks, peak_src, clk, e4m3_peak):
 
 
 def measure_extra(name, args, dev, local, peaks, peak_src, e4m3_peak):
-    """Device-side figures of a second workload in the same run (the e4m3 128K layer beside
-    the bf16 one): stage times, work and roofline, timed as the main workload is."""
+    """Device-side figures of another workload in the same run (the e4m3 and the multi-head
+    128K layers beside the bf16 one): stage times, work and roofline, timed as the main
+    workload is."""
     w = S.WORKLOADS[name]
     inp = S.make_inputs(name)
     layer = Layer(inp, dev)
@@ -478,7 +481,7 @@ def run_native(args, world, rank, local):
     alg, executed, density = work_counts(w, cnt, idx)
     pool_bytes, pm_bytes = pool_mask_bytes(w)
     extra_names = ([] if (args.no_extra or world > 1 or w.name != "llama128k")
-                   else ["fp8_128k"])
+                   else ["fp8_128k", "mha128k"])
     e4m3_peak = None
     if w.dtype == "e4m3" or extra_names:
         e4m3_peak = measure_e4m3_peak(dev)
@@ -611,7 +614,8 @@ def main():
                     help="N > 1: independent layers per rank (replicas, weak scaling) or one "
                          "layer split by KV-head group (heads, strong scaling; no exchange)")
     ap.add_argument("--no-extra", action="store_true",
-                    help="skip the e4m3 128K layer that the default bf16 128K run also times")
+                    help="skip the e4m3 and multi-head 128K layers that the default bf16 128K "
+                         "run also times")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     try:
