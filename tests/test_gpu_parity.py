@@ -326,6 +326,29 @@ def test_full_size_workloads(name, cuda_device):
     _full_size(name, cuda_device)
 
 
+@pytest.mark.parametrize("name", ["llama128k", "fp8_128k"])
+def test_query_block_pairing_at_full_size(name, cuda_device):
+    """The general work split (two neighbouring query blocks of one head per CTA, forced with
+    FP_PAIR_QBLOCKS) on the full 128K GQA layers: the same output, bit for bit, as the default
+    head-pair split that the full-size oracle comparison checks (16,384 CTAs, kept lists up to
+    ~80 blocks per row)."""
+    inp = S.make_inputs(name)
+    w = inp.workload
+    q, k, v, sc = device_inputs(inp, cuda_device)
+    kw = dict(q_scale=sc["q_scale"], k_scale=sc["k_scale"], v_scale=sc["v_scale"],
+              return_lse=True)
+    b = _batch(inp, cuda_device)
+    qp, kp = fp.pool_qk(q, k, w.block, batch=b, q_scale=sc["q_scale"], k_scale=sc["k_scale"])
+    _, cnt, idx = fp.build_block_mask(qp, kp, w.alpha, block=w.block, batch=b, mask_bits=False)
+    out, lse = fp.sparse_prefill_attn(q, k, v, cnt, idx, w.block, batch=b, **kw)
+    T = q.shape[0]
+    cb = fp.ChunkedBatch.make((T,), (T,), w.block, cuda_device)
+    out_q, lse_q = fp.sparse_prefill_attn_chunked(q, k, v, cnt, idx, cb, pair_qblocks=True, **kw)
+    fp.check_status(cuda_device)
+    assert torch.equal(out, out_q)
+    assert torch.equal(lse, lse_q)
+
+
 def test_longest_sequence_512k(cuda_device):
     """One 524,288-token sequence (4,096 blocks per row): the largest single layer the tests
     run. Pooled means and the mask against the oracle in full, the attention on sampled rows."""
